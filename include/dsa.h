@@ -1,0 +1,175 @@
+/*
+ * dsa.h — C ABI of a B200 (sm_100a) implementation of DeepSeek Sparse
+ * Attention (DSA): lightning indexer -> per-query top-k -> softmax attention
+ * of H query heads over only the kept keys of one MQA-shared K/V.
+ *
+ * What is computed follows the DeepSeek Sparse Attention page
+ * (kwkr.cn/news/60693):
+ *   section 3.2  lightning indexer: I = relu(matmul(q_idx, k_idx^T) * scale),
+ *                scale = index_dim^-0.5, FP8 inputs in a low index dimension;
+ *   section 3.3  fine-grained token selection: each query keeps its top-k
+ *                keys, then ordinary softmax attention runs over those keys;
+ *   section 4.1  precision: FP8 index stage, BF16 attention stage;
+ *   section 4.2  memory: all query heads share one K/V (MQA); rows are laid
+ *                out on 128-byte boundaries;
+ *   section 7.2  per-length settings (FP8 at 32K/64K, BF16 index at 128K).
+ * Readings where the page is silent (stated once here, used everywhere):
+ *   - causal: query t sees keys s <= t, the diagonal included;
+ *   - the indexer score of a pair is fp32(fp32(q.k) * scale), then ReLU maps
+ *     every non-positive score (and -0) to +0;
+ *   - order: keys are ranked by (score descending, key index ascending), so
+ *     ties go to the lower key index; a query keeps min(top_k, t+1) keys;
+ *   - indices[t] lists the kept keys in that rank order and pads with -1;
+ *   - attention softmax scale defaults to D^-0.5; output is BF16 (nearest).
+ *
+ * Conventions for every call:
+ *   - Pointers marked "device" are CUDA device pointers on the current
+ *     device; the caller owns every buffer.  No call allocates memory.
+ *   - Tensors are dense row-major.  Device pointers must be 16-byte aligned;
+ *     128-byte alignment is recommended (row starts then fall on 128 B).
+ *   - `stream` is a cudaStream_t passed as void*.  Calls only enqueue work;
+ *     they are asynchronous and keep no state between calls, so calls on
+ *     distinct workspaces may run concurrently.
+ *   - Argument errors are reported synchronously by the return value and
+ *     nothing is enqueued.  Errors found on the device (a bounded wait that
+ *     ran out) are recorded in a per-device status word that
+ *     dsa_sync_status() reads and clears.
+ *   - idx_scale / attn_scale: pass NaN to use index_dim^-0.5 / D^-0.5
+ *     (each rounded to float32).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, size out of range  */
+  DSA_ERR_UNSUPPORTED = 2,  /* shape the kernels do not handle              */
+  DSA_ERR_WORKSPACE = 3,    /* workspace smaller than *_workspace_size()    */
+  DSA_ERR_CUDA = 4,         /* a CUDA runtime call failed                   */
+  DSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out           */
+  DSA_ERR_DEVICE = 6        /* other device-side fault recorded by a kernel */
+} dsa_status;
+
+typedef enum {
+  DSA_IDX_FP8_E4M3 = 0,     /* OCP FP8 E4M3 bytes                            */
+  DSA_IDX_BF16 = 1          /* bfloat16                                      */
+} dsa_idx_dtype;
+
+/* Limits of this implementation. */
+#define DSA_MAX_TOP_K 2048
+#define DSA_MAX_INDEX_DIM 256
+#define DSA_MAX_HEADS 16
+
+/* Human-readable name of a status code (static string). */
+const char* dsa_status_string(dsa_status s);
+
+/* Library version as "major.minor.patch" (static string). */
+const char* dsa_version(void);
+
+/*
+ * dsa_indexer_scores — the lightning indexer of section 3.2 exactly as the
+ * page's snippet writes it: the dense matrix
+ *     scores[t, s] = relu(fp32(q_idx[t] . k_idx[s]) * idx_scale)
+ * for t < Lq, s < Lk, with no causal mask and no selection.  Runs on the same
+ * tcgen05 tensor-core tiles as dsa_prefill.  Meant for checking and small
+ * sizes: it writes Lq*Lk floats.
+ *   q_idx   device [Lq, d_idx]   FP8 E4M3 or BF16 (idx_dtype)
+ *   k_idx   device [Lk, d_idx]
+ *   scores  device [Lq, Lk] float32, written
+ * d_idx must be a multiple of 32 bytes of the element type and <= 256.
+ * Returns DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED on bad arguments.
+ */
+dsa_status dsa_indexer_scores(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                              float idx_scale, int64_t Lq, int64_t Lk, float* scores,
+                              void* stream);
+
+/* Bytes of device workspace dsa_prefill needs for these sizes. */
+size_t dsa_prefill_workspace_size(int64_t L, int d_idx, int idx_dtype, int H, int D, int top_k);
+
+/*
+ * dsa_prefill — DSA over one causal sequence of length L (sections 3.1-3.3,
+ * 4.1-4.3): indexer scores of every causal pair, per-query top-k, then
+ * softmax attention of H heads over the kept keys.  The L x L score matrix
+ * is never written to memory.
+ *   q_idx, k_idx  device [L, d_idx]  FP8 E4M3 or BF16 (idx_dtype); d_idx a
+ *                 multiple of 32 bytes of the element type, <= 256
+ *   Q             device [L, H, D] BF16 (query heads)
+ *   K, V          device [L, D]    BF16 (one K/V shared by all heads)
+ *   indices       device [L, top_k] int32, written: kept keys of query t in
+ *                 rank order, -1 padded (t+1 < top_k)
+ *   O             device [L, H, D] BF16, written
+ *   workspace     device, >= dsa_prefill_workspace_size(...) bytes, 256-byte
+ *                 aligned; contents on entry are ignored
+ * Limits: 1 <= top_k <= 2048, 1 <= H <= 16, D in {64, 128}, L >= 1.
+ */
+dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                       float idx_scale, const void* Q, const void* K, const void* V, int64_t L,
+                       int H, int D, float attn_scale, int top_k, int32_t* indices, void* O,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace dsa_decode needs.  total_rows = sum of lengths. */
+size_t dsa_decode_workspace_size(int B, int64_t total_rows, int d_idx, int idx_dtype, int H,
+                                 int D, int top_k);
+
+/*
+ * dsa_decode — one decode step for a batch of B cached sequences (the same
+ * three stages as dsa_prefill for one new query per sequence; the indexer
+ * scan streams the cache, section 4.2).  The cache is ragged and contiguous
+ * per sequence: rows seq_start[b] .. seq_start[b+1]-1 belong to sequence b.
+ * The new token's rows are already in the cache, so the query of sequence b
+ * sits at position len_b - 1 and sees all len_b rows.
+ *   k_idx      device [total_rows, d_idx] FP8 E4M3 or BF16
+ *   K, V       device [total_rows, D] BF16
+ *   seq_start  device [B+1] int64, nondecreasing, seq_start[0] = 0,
+ *              seq_start[B] = total_rows; every length >= 1
+ *   q_idx      device [B, d_idx];  Q device [B, H, D] BF16
+ *   O          device [B, H, D] BF16, written
+ *   indices    device [B, top_k] int32, written when non-null (rank order,
+ *              -1 padded), positions relative to the sequence's first row
+ *   max_len    host bound on every len_b (sizes the scan grid)
+ * Limits as dsa_prefill; max_len <= 2^31 - 1.
+ */
+dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int64_t* seq_start,
+                      int B, int64_t total_rows, int64_t max_len, int idx_dtype, int d_idx, int D,
+                      const void* q_idx, const void* Q, int H, int top_k, float idx_scale,
+                      float attn_scale, void* O, int32_t* indices, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * dsa_sync_status — synchronise `stream`, then read and clear the current
+ * device's status word (the first device-side error since the last read).
+ * Returns DSA_OK when no kernel recorded an error, DSA_ERR_CUDA when the
+ * synchronisation itself failed.
+ */
+dsa_status dsa_sync_status(void* stream);
+
+/*
+ * dsa_last_stats — host copy of counters the last dsa_prefill/dsa_decode
+ * call left in `workspace` (synchronises `stream`):
+ *   out[0] rows that took the exact fallback select, out[1] rows whose
+ *   candidate list overflowed, out[2] total candidates emitted.
+ * Diagnostic only.
+ */
+dsa_status dsa_last_stats(const void* workspace, int64_t out[4], void* stream);
+
+/*
+ * dsa_debug_wait_timeout — runs one tiny kernel whose only work is a
+ * bounded wait on a shared-memory barrier that nothing completes, with a
+ * limit of `limit_ns` nanoseconds.  The kernel records DSA_ERR_TIMEOUT in the
+ * status word and returns normally, so the context stays usable.  Exists to
+ * test the timeout path without hanging or faulting a GPU.
+ */
+dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

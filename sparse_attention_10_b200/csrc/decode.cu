@@ -1,0 +1,318 @@
+// Decode step: indexer scan over the cache and per-sequence top-k (sm_100a).
+//
+// One new query per sequence attends over that sequence's cached rows (the
+// DeepSeek Sparse Attention page, kwkr.cn/news/60693, sections 3.2-3.3; the
+// scan streams the index cache once, section 4.2).
+//
+// decode_scan_kernel: grid (chunks, B).  Each thread scores whole cache rows:
+// 16-byte loads of the row, FP32 FMA in index order (exact for integer
+// inputs), relu(fp32(dot) * scale) into a score array, plus a shared-memory
+// histogram of the top 11 bits of each score, added to a per-sequence
+// histogram in global memory.
+//
+// decode_select_kernel: one CTA per sequence.  The histogram gives the bin of
+// the m-th best score; every key at or above that bin is compacted into shared
+// memory (or, when too many, into a global scratch row) and the exact select
+// plus sort of the prefill path finishes the row.
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsa {
+
+// Shared with select.cu (same translation-unit-free helpers re-declared here).
+namespace {
+
+constexpr int kScanThreads = 256;
+constexpr int kScanRowsPerCta = 4096;
+constexpr int kHistBins = 2048;           // score bits 30..20 (scores are >= +0)
+constexpr int kSelThreads = 1024;
+constexpr int kSmemKeys = 12288;          // candidates held in shared memory
+
+__device__ __forceinline__ unsigned long long score_key(float sc, uint32_t s) {
+  return (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xFFFFFFFFu - s);
+}
+
+template <int ESIZE>
+__device__ __forceinline__ float dot_row(const float* q, const void* base, int64_t row, int d) {
+  float acc = 0.0f;
+  if (ESIZE == 1) {
+    const uint8_t* r = static_cast<const uint8_t*>(base) + row * d;
+    for (int j = 0; j < d; j += 16) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(r + j));
+      const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const __nv_fp8x2_storage_t pair =
+              static_cast<__nv_fp8x2_storage_t>((words[u] >> (16 * h)) & 0xFFFFu);
+          const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+          acc = fmaf(q[j + 4 * u + 2 * h], f.x, acc);
+          acc = fmaf(q[j + 4 * u + 2 * h + 1], f.y, acc);
+        }
+      }
+    }
+  } else {
+    const __nv_bfloat16* r = static_cast<const __nv_bfloat16*>(base) + row * d;
+    for (int j = 0; j < d; j += 8) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(r + j));
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 f = __bfloat1622float2(h2[u]);
+        acc = fmaf(q[j + 2 * u], f.x, acc);
+        acc = fmaf(q[j + 2 * u + 1], f.y, acc);
+      }
+    }
+  }
+  return acc;
+}
+
+// seq_start must start at 0, end at total_rows, and give lengths in [1, max_len].
+__global__ void validate_kernel(const int64_t* seq_start, int B, int64_t total_rows,
+                                int64_t max_len, int* invalid) {
+  bool bad = false;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t len = seq_start[b + 1] - seq_start[b];
+    bad |= len < 1 || len > max_len;
+  }
+  if (threadIdx.x == 0) bad |= seq_start[0] != 0 || seq_start[B] != total_rows;
+  if (__syncthreads_or(bad) && threadIdx.x == 0) {
+    *invalid = 1;
+    record_error(DSA_ERR_INVALID_ARG);
+  }
+}
+
+struct ScanParams {
+  const void* k_idx;
+  const void* q_idx;
+  int d;
+  const int64_t* seq_start;
+  float scale;
+  float* scores;
+  unsigned int* hist;
+  const int* invalid;
+};
+
+template <int ESIZE>
+__global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanParams p) {
+  __shared__ float qf[DSA_MAX_INDEX_DIM];
+  __shared__ unsigned int hist[kHistBins];
+  if (*p.invalid) return;
+  const int b = blockIdx.y;
+  const int64_t base = p.seq_start[b];
+  const int64_t len = p.seq_start[b + 1] - base;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kScanRowsPerCta;
+  if (c0 >= len) return;
+  const int64_t c1 = min64(len, c0 + kScanRowsPerCta);
+  for (int j = threadIdx.x; j < p.d; j += blockDim.x) {
+    if (ESIZE == 1) {
+      const __nv_fp8_storage_t v = static_cast<const __nv_fp8_storage_t*>(p.q_idx)[b * p.d + j];
+      qf[j] = __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)));
+    } else {
+      qf[j] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q_idx)[b * p.d + j]);
+    }
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  for (int64_t s = c0 + threadIdx.x; s < c1; s += blockDim.x) {
+    float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, base + s, p.d), p.scale);
+    sc = sc > 0.0f ? sc : 0.0f;
+    p.scores[base + s] = sc;
+    atomicAdd(&hist[__float_as_uint(sc) >> 20], 1u);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(&p.hist[static_cast<int64_t>(b) * kHistBins + i], hist[i]);
+}
+
+// ---- select ------------------------------------------------------------------
+
+__device__ __forceinline__ void find_from_top_256(const unsigned int* hist, int R, int* out) {
+  const int lane = threadIdx.x & 31;
+  unsigned int local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) local += hist[255 - 8 * lane - i];
+  unsigned int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const unsigned int ballot = __ballot_sync(0xFFFFFFFFu, incl >= static_cast<unsigned int>(R));
+  const int src = __ffs(ballot) - 1;
+  if (lane == src) {
+    unsigned int run = incl - local;
+    for (int i = 0; i < 8; ++i) {
+      const int bb = 255 - 8 * lane - i;
+      if (run + hist[bb] >= static_cast<unsigned int>(R)) {
+        out[0] = bb;
+        out[1] = R - static_cast<int>(run);
+        break;
+      }
+      run += hist[bb];
+    }
+  }
+}
+
+template <typename KeyPtr>
+__device__ unsigned long long radix_select(KeyPtr keys, int n, int R, unsigned int* hist,
+                                           int* sh) {
+  unsigned long long prefix = 0, mask = 0;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long k = keys[i];
+      if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) find_from_top_256(hist, R, sh);
+    __syncthreads();
+    const int bsel = sh[0];
+    R = sh[1];
+    prefix |= static_cast<unsigned long long>(bsel) << shift;
+    mask |= 0xFFull << shift;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+__device__ void bitonic_desc(unsigned long long* a, int P) {
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < P / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool desc = (lo & size) == 0;
+        const unsigned long long x = a[lo], y = a[hi];
+        if ((x < y) == desc) {
+          a[lo] = y;
+          a[hi] = x;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+struct DSelParams {
+  const float* scores;
+  const unsigned int* hist;
+  const int64_t* seq_start;
+  int top_k;
+  int32_t* indices;
+  unsigned long long* scratch;   // [total_rows] (rows of sequence b at seq_start[b])
+  const int* invalid;
+};
+
+__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelParams p) {
+  extern __shared__ unsigned long long ds_smem[];
+  unsigned long long* keys = ds_smem;                       // [kSmemKeys]
+  unsigned long long* sel = keys + kSmemKeys;               // [2048]
+  unsigned int* h256 = reinterpret_cast<unsigned int*>(sel + DSA_MAX_TOP_K);
+  int* sh = reinterpret_cast<int*>(h256 + 256);             // [8]
+  if (*p.invalid) return;
+  const int b = blockIdx.x;
+  const int64_t base = p.seq_start[b];
+  const int n = static_cast<int>(p.seq_start[b + 1] - base);
+  const int m = min(p.top_k, n);
+  const float* sc = p.scores + base;
+  const unsigned int* hist = p.hist + static_cast<int64_t>(b) * kHistBins;
+
+  // Bin of the m-th best score (bins scanned from the top by warp 0).
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    unsigned int local = 0;
+    for (int i = 0; i < kHistBins / 32; ++i) local += hist[kHistBins - 1 - (kHistBins / 32) * lane - i];
+    unsigned int incl = local;
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned int ballot = __ballot_sync(0xFFFFFFFFu, incl >= static_cast<unsigned int>(m));
+    const int src = __ffs(ballot) - 1;
+    if (lane == src) {
+      unsigned int run = incl - local;
+      for (int i = 0; i < kHistBins / 32; ++i) {
+        const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
+        run += hist[bb];
+        if (run >= static_cast<unsigned int>(m)) {
+          sh[0] = bb;
+          sh[1] = static_cast<int>(run);  // keys in bins >= bb
+          break;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t bin = static_cast<uint32_t>(sh[0]);
+  const int ncand = sh[1];
+  __syncthreads();
+
+  unsigned long long* cand;
+  if (ncand <= kSmemKeys) {
+    cand = keys;
+  } else {
+    cand = p.scratch + base;
+  }
+  if (threadIdx.x == 0) sh[2] = 0;
+  __syncthreads();
+  for (int s = threadIdx.x; s < n; s += blockDim.x) {
+    const float v = sc[s];
+    if ((__float_as_uint(v) >> 20) >= bin) {
+      const int pos = atomicAdd(&sh[2], 1);
+      if (pos < ncand) cand[pos] = score_key(v, s);
+    }
+  }
+  __syncthreads();
+  const unsigned long long kth = ncand > m ? radix_select(cand, ncand, m, h256, sh) : 0ull;
+  if (threadIdx.x == 0) sh[3] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < ncand; i += blockDim.x) {
+    const unsigned long long k = cand[i];
+    if (k >= kth) {
+      const int pos = atomicAdd(&sh[3], 1);
+      if (pos < m) sel[pos] = k;
+    }
+  }
+  int P = 2;
+  while (P < m) P <<= 1;
+  __syncthreads();
+  for (int i = m + threadIdx.x; i < P; i += blockDim.x) sel[i] = 0ull;
+  bitonic_desc(sel, P);
+  for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
+    p.indices[static_cast<int64_t>(b) * p.top_k + i] =
+        i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
+}
+
+}  // namespace
+
+dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
+  if (cudaMemsetAsync(a.hist, 0, sizeof(unsigned int) * kHistBins * a.B, stream) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.invalid);
+  ScanParams sp{a.k_idx, a.q_idx, a.d, a.seq_start, a.scale, a.scores, a.hist, a.invalid};
+  const dim3 grid(static_cast<unsigned int>((a.max_len + kScanRowsPerCta - 1) / kScanRowsPerCta),
+                  static_cast<unsigned int>(a.B));
+  if (a.esize == 1)
+    decode_scan_kernel<1><<<grid, kScanThreads, 0, stream>>>(sp);
+  else
+    decode_scan_kernel<2><<<grid, kScanThreads, 0, stream>>>(sp);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+
+  DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid};
+  const size_t smem = static_cast<size_t>(kSmemKeys + DSA_MAX_TOP_K) * 8 + 256 * 4 + 32;
+  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  decode_select_kernel<<<a.B, kSelThreads, smem, stream>>>(dp);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace dsa

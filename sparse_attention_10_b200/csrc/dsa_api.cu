@@ -1,0 +1,375 @@
+// C ABI of the DSA library: argument checks, workspace layout, launch order.
+//
+// dsa_prefill runs, in stream order:
+//   1. indexer (sample mode)  scores against a few key tiles per query tile;
+//   2. tau_kernel             per-row raw-accumulator threshold from the sample;
+//   3. indexer (filter mode)  every causal score, candidates >= threshold;
+//   4. select_kernel          exact top-k + order per row (fallback queue);
+//      fallback_kernel        exact recomputation for queued rows;
+//   5. attn_kernel            gathered sparse MQA attention.
+// dsa_decode runs the scan, the per-sequence select and split attention.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsa {
+
+__device__ unsigned int g_status = 0;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int esize_of(int idx_dtype) {
+  return idx_dtype == DSA_IDX_FP8_E4M3 ? 1 : (idx_dtype == DSA_IDX_BF16 ? 2 : 0);
+}
+
+dsa_status check_index_dims(int idx_dtype, int d_idx) {
+  const int es = esize_of(idx_dtype);
+  if (es == 0) return DSA_ERR_INVALID_ARG;
+  if (d_idx <= 0 || d_idx > DSA_MAX_INDEX_DIM) return DSA_ERR_INVALID_ARG;
+  if ((d_idx * es) % 32 != 0) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+float default_scale(float s, int dim) {
+  return std::isnan(s) ? static_cast<float>(1.0 / std::sqrt(static_cast<double>(dim))) : s;
+}
+
+// ---- prefill workspace ----------------------------------------------------------
+
+struct PrefillPlan {
+  int cap_half;     // candidates kept per (row, column half)
+  int cap_all;      // rows with t + 1 <= cap_all keep every key
+  int target;       // candidates aimed for per row by the threshold
+  int samp_ld;
+  int fb_ctas;
+  size_t off_counters, off_tau, off_cand_n, off_cand, off_samp, off_fb_rows, off_fb_scratch, total;
+};
+
+PrefillPlan plan_prefill(int64_t L, int top_k) {
+  PrefillPlan p{};
+  p.target = (top_k * 17 + 9) / 10;                      // 1.7 k
+  p.cap_half = ((top_k * 5 / 4 + 128) + 15) / 16 * 16;    // per half: 1.25 k + 128
+  p.cap_all = p.cap_half;  // rows kept whole must fit one column half
+  p.samp_ld = kSampTilesMax * kBN;
+  p.fb_ctas = std::max(1, num_sms());
+  size_t o = 0;
+  p.off_counters = o;
+  o = align_up(o + 64 * sizeof(int));
+  p.off_tau = o;
+  o = align_up(o + L * sizeof(float));
+  p.off_cand_n = o;
+  o = align_up(o + 2 * L * sizeof(int));
+  p.off_cand = o;
+  o = align_up(o + static_cast<size_t>(2 * L) * p.cap_half * sizeof(unsigned long long));
+  p.off_samp = o;
+  o = align_up(o + static_cast<size_t>(L) * p.samp_ld * sizeof(uint16_t));
+  p.off_fb_rows = o;
+  o = align_up(o + L * sizeof(int));
+  p.off_fb_scratch = o;
+  o = align_up(o + static_cast<size_t>(p.fb_ctas) * L * sizeof(unsigned long long));
+  p.total = o;
+  return p;
+}
+
+// ---- decode workspace -------------------------------------------------------------
+
+constexpr int kDecodeSplits = 8;
+
+struct DecodePlan {
+  size_t off_counters, off_scores, off_hist, off_keys, off_indices, off_part, total;
+};
+
+DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k) {
+  DecodePlan p{};
+  size_t o = 0;
+  p.off_counters = o;
+  o = align_up(o + 64 * sizeof(int));
+  p.off_scores = o;
+  o = align_up(o + total_rows * sizeof(float));
+  p.off_hist = o;
+  o = align_up(o + static_cast<size_t>(B) * 2048 * sizeof(unsigned int));
+  p.off_keys = o;
+  o = align_up(o + total_rows * sizeof(unsigned long long));
+  p.off_indices = o;
+  o = align_up(o + static_cast<size_t>(B) * top_k * sizeof(int32_t));
+  p.off_part = o;
+  o = align_up(o + static_cast<size_t>(B) * kDecodeSplits * H * (D + 2) * sizeof(float));
+  p.total = o;
+  return p;
+}
+
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, limit_ns, nullptr);  // nothing arrives
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_arrive(smem_u32(&bar));  // leave the barrier complete
+}
+
+}  // namespace
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+uint64_t wait_limit_ns() { return 2000000000ull; }  // 2 s per wait
+
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_WORKSPACE: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA runtime error";
+    case DSA_ERR_TIMEOUT: return "device-side wait timed out";
+    case DSA_ERR_DEVICE: return "device-side error";
+  }
+  return "unknown status";
+}
+
+const char* dsa_version(void) { return "0.1.0"; }
+
+dsa_status dsa_indexer_scores(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                              float idx_scale, int64_t Lq, int64_t Lk, float* scores,
+                              void* stream) {
+  if (!q_idx || !k_idx || !scores || Lq < 1 || Lk < 1) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (Lq > (int64_t(1) << 31) - 1 || Lk > (int64_t(1) << 31) - 1) return DSA_ERR_UNSUPPORTED;
+  dsa_status st = check_index_dims(idx_dtype, d_idx);
+  if (st != DSA_OK) return st;
+  IndexerLaunch a{};
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.esize = esize_of(idx_dtype);
+  a.d = d_idx;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.scale = default_scale(idx_scale, d_idx);
+  a.mode = kModeDense;
+  a.scores = scores;
+  a.limit_ns = wait_limit_ns();
+  return launch_indexer(a, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_prefill_workspace_size(int64_t L, int d_idx, int idx_dtype, int H, int D, int top_k) {
+  (void)d_idx; (void)idx_dtype; (void)H; (void)D;
+  if (L < 1 || top_k < 1) return 0;
+  return plan_prefill(L, top_k).total;
+}
+
+dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                       float idx_scale, const void* Q, const void* K, const void* V, int64_t L,
+                       int H, int D, float attn_scale, int top_k, int32_t* indices, void* O,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q_idx || !k_idx || !Q || !K || !V || !indices || !O || !workspace) return DSA_ERR_INVALID_ARG;
+  for (const void* ptr : {q_idx, k_idx, Q, K, V, static_cast<const void*>(indices),
+                          static_cast<const void*>(O)})
+    if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return DSA_ERR_INVALID_ARG;
+  if (L < 1 || L > (int64_t(1) << 31) - 1) return DSA_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
+  if (H < 1 || H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
+  dsa_status st = check_index_dims(idx_dtype, d_idx);
+  if (st != DSA_OK) return st;
+  const PrefillPlan plan = plan_prefill(L, top_k);
+  if (workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* counters = reinterpret_cast<int*>(ws + plan.off_counters);
+  float* tau = reinterpret_cast<float*>(ws + plan.off_tau);
+  int* cand_n = reinterpret_cast<int*>(ws + plan.off_cand_n);
+  unsigned long long* cand = reinterpret_cast<unsigned long long*>(ws + plan.off_cand);
+  uint16_t* samp = reinterpret_cast<uint16_t*>(ws + plan.off_samp);
+  int* fb_rows = reinterpret_cast<int*>(ws + plan.off_fb_rows);
+  unsigned long long* fb_scratch = reinterpret_cast<unsigned long long*>(ws + plan.off_fb_scratch);
+  const int es = esize_of(idx_dtype);
+  const float iscale = default_scale(idx_scale, d_idx);
+  const float ascale = default_scale(attn_scale, D);
+
+  if (cudaMemsetAsync(counters, 0, 64 * sizeof(int), s) != cudaSuccess) return DSA_ERR_CUDA;
+
+  IndexerLaunch a{};
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.esize = es;
+  a.d = d_idx;
+  a.Lq = L;
+  a.Lk = L;
+  a.scale = iscale;
+  a.limit_ns = wait_limit_ns();
+  if (L > plan.cap_all) {
+    a.mode = kModeSample;
+    a.samp = samp;
+    a.samp_ld = plan.samp_ld;
+    a.cap = plan.cap_all;
+    if ((st = launch_indexer(a, s)) != DSA_OK) return st;
+  }
+  if ((st = launch_tau_select(samp, plan.samp_ld, L, plan.cap_all, plan.target, iscale, tau, s)) !=
+      DSA_OK)
+    return st;
+  a.mode = kModeFilter;
+  a.tau = tau;
+  a.cand = cand;
+  a.cand_n = cand_n;
+  a.cap = plan.cap_half;
+  if ((st = launch_indexer(a, s)) != DSA_OK) return st;
+
+  SelectLaunch sl{};
+  sl.L = L;
+  sl.top_k = top_k;
+  sl.cap = plan.cap_half;
+  sl.cand = cand;
+  sl.cand_n = cand_n;
+  sl.indices = indices;
+  sl.fb_rows = fb_rows;
+  sl.counters = counters;
+  sl.q_idx = q_idx;
+  sl.k_idx = k_idx;
+  sl.esize = es;
+  sl.d = d_idx;
+  sl.scale = iscale;
+  sl.fb_scratch = fb_scratch;
+  sl.fb_ctas = plan.fb_ctas;
+  if ((st = launch_select(sl, s)) != DSA_OK) return st;
+
+  AttnLaunch at{};
+  at.Q = static_cast<const __nv_bfloat16*>(Q);
+  at.K = static_cast<const __nv_bfloat16*>(K);
+  at.V = static_cast<const __nv_bfloat16*>(V);
+  at.idx = indices;
+  at.ld_idx = top_k;
+  at.nq = L;
+  at.H = H;
+  at.D = D;
+  at.scale_log2 = ascale * 1.4426950408889634f;
+  at.top_k = top_k;
+  at.seq_start = nullptr;
+  at.nsplit = 1;
+  at.O = static_cast<__nv_bfloat16*>(O);
+  return launch_attention(at, s);
+}
+
+size_t dsa_decode_workspace_size(int B, int64_t total_rows, int d_idx, int idx_dtype, int H,
+                                 int D, int top_k) {
+  (void)d_idx; (void)idx_dtype;
+  if (B < 1 || total_rows < 1 || H < 1 || top_k < 1) return 0;
+  return plan_decode(B, total_rows, H, D, top_k).total;
+}
+
+dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int64_t* seq_start,
+                      int B, int64_t total_rows, int64_t max_len, int idx_dtype, int d_idx, int D,
+                      const void* q_idx, const void* Q, int H, int top_k, float idx_scale,
+                      float attn_scale, void* O, int32_t* indices, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!k_idx || !K || !V || !seq_start || !q_idx || !Q || !O || !workspace)
+    return DSA_ERR_INVALID_ARG;
+  for (const void* ptr : {k_idx, K, V, q_idx, Q, static_cast<const void*>(O)})
+    if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
+  if (indices && !aligned16(indices)) return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_start) & 7) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (B < 1 || total_rows < 1 || max_len < 1 || max_len > (int64_t(1) << 31) - 1)
+    return DSA_ERR_INVALID_ARG;
+  if (top_k < 1 || top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
+  if (H < 1 || H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
+  dsa_status st = check_index_dims(idx_dtype, d_idx);
+  if (st != DSA_OK) return st;
+  const DecodePlan plan = plan_decode(B, total_rows, H, D, top_k);
+  if (workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* idx = indices ? indices : reinterpret_cast<int32_t*>(ws + plan.off_indices);
+  if (cudaMemsetAsync(ws + plan.off_counters, 0, 64 * sizeof(int), s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+
+  DecodeLaunch dl{};
+  dl.k_idx = k_idx;
+  dl.q_idx = q_idx;
+  dl.esize = esize_of(idx_dtype);
+  dl.d = d_idx;
+  dl.seq_start = seq_start;
+  dl.B = B;
+  dl.total_rows = total_rows;
+  dl.max_len = max_len;
+  dl.scale = default_scale(idx_scale, d_idx);
+  dl.top_k = top_k;
+  dl.scores = reinterpret_cast<float*>(ws + plan.off_scores);
+  dl.hist = reinterpret_cast<unsigned int*>(ws + plan.off_hist);
+  dl.indices = idx;
+  dl.keys = reinterpret_cast<unsigned long long*>(ws + plan.off_keys);
+  dl.invalid = reinterpret_cast<int*>(ws + plan.off_counters) + 8;
+  if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
+
+  AttnLaunch at{};
+  at.Q = static_cast<const __nv_bfloat16*>(Q);
+  at.K = static_cast<const __nv_bfloat16*>(K);
+  at.V = static_cast<const __nv_bfloat16*>(V);
+  at.idx = idx;
+  at.ld_idx = top_k;
+  at.nq = B;
+  at.H = H;
+  at.D = D;
+  at.scale_log2 = default_scale(attn_scale, D) * 1.4426950408889634f;
+  at.top_k = top_k;
+  at.seq_start = seq_start;
+  at.nsplit = kDecodeSplits;
+  at.O = static_cast<__nv_bfloat16*>(O);
+  at.part = reinterpret_cast<float*>(ws + plan.off_part);
+  at.invalid = dl.invalid;
+  return launch_attention(at, s);
+}
+
+dsa_status dsa_sync_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return DSA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return static_cast<dsa_status>(v);
+}
+
+dsa_status dsa_last_stats(const void* workspace, int64_t out[4], void* stream) {
+  if (!workspace || !out) return DSA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  int c[4] = {0, 0, 0, 0};
+  if (cudaMemcpy(c, workspace, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) out[i] = c[i];
+  return DSA_OK;
+}
+
+dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,116 @@
+// Host-side declarations shared by the DSA translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dsa.h"
+
+namespace dsa {
+
+// ---- indexer (tcgen05) -------------------------------------------------------
+
+enum IndexerMode { kModeDense = 0, kModeSample = 1, kModeFilter = 2 };
+
+constexpr int kBM = 128;          // query rows per tile = TMEM lanes
+constexpr int kBN = 256;          // keys per tile = TMEM columns per accumulator
+constexpr int kSampTilesMax = 16; // key tiles sampled per query tile for the threshold
+
+struct IndexerLaunch {
+  const void* q_idx;
+  const void* k_idx;
+  int esize;          // 1 = FP8 E4M3, 2 = BF16
+  int d;              // index dim (elements)
+  int64_t Lq, Lk;
+  float scale;
+  int mode;
+  // filter
+  const float* tau;
+  unsigned long long* cand;
+  int* cand_n;
+  int cap;
+  // sample
+  uint16_t* samp;
+  int samp_ld;
+  // dense
+  float* scores;
+  uint64_t limit_ns;
+};
+
+dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream);
+
+// Threshold per query row from the sampled scores (raw accumulator domain).
+dsa_status launch_tau_select(const uint16_t* samp, int samp_ld, int64_t L, int cap, int target,
+                             float scale, float* tau, cudaStream_t stream);
+
+// ---- select -------------------------------------------------------------------
+
+struct SelectLaunch {
+  int64_t L;
+  int top_k;
+  int cap;
+  const unsigned long long* cand;
+  const int* cand_n;
+  int32_t* indices;
+  int* fb_rows;          // [L] rows that need the exact fallback
+  int* counters;         // [0] fallback rows, [1] overflow rows, [2] candidates
+  // fallback inputs
+  const void* q_idx;
+  const void* k_idx;
+  int esize, d;
+  float scale;
+  unsigned long long* fb_scratch;  // [fb_ctas, L]
+  int fb_ctas;
+};
+
+dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream);
+
+// ---- attention ---------------------------------------------------------------
+
+struct AttnLaunch {
+  const __nv_bfloat16* Q;      // [nq, H, D]
+  const __nv_bfloat16* K;      // [rows, D]
+  const __nv_bfloat16* V;
+  const int32_t* idx;          // [nq, ld_idx]
+  int ld_idx;
+  int64_t nq;
+  int H, D;
+  float scale_log2;            // softmax scale * log2(e)
+  int top_k;
+  // prefill: count(q) = min(top_k, q + 1), row base 0
+  // decode:  count(q) = min(top_k, len_q), row base seq_start[q]
+  const int64_t* seq_start;    // null for prefill
+  int nsplit;                  // splits of the key list per query (1 = final output)
+  __nv_bfloat16* O;            // [nq, H, D] (nsplit == 1)
+  float* part;                 // [nq, nsplit, H, D + 2] (nsplit > 1)
+  const int* invalid;          // nonzero: skip all work (decode inputs failed validation)
+};
+
+dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream);
+
+// ---- decode ------------------------------------------------------------------
+
+struct DecodeLaunch {
+  const void* k_idx;
+  const void* q_idx;
+  int esize, d;
+  const int64_t* seq_start;
+  int B;
+  int64_t total_rows, max_len;
+  float scale;
+  int top_k;
+  float* scores;               // [total_rows]
+  unsigned int* hist;          // [B, 4096]
+  int32_t* indices;            // [B, top_k]
+  unsigned long long* keys;    // [total_rows] scratch (many-candidate rows)
+  int* invalid;                // set when seq_start fails validation
+};
+
+dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream);
+
+int num_sms();
+uint64_t wait_limit_ns();
+
+}  // namespace dsa

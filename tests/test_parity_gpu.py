@@ -1,0 +1,252 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Bar: indices bit-exact (integer-valued indexer inputs make every score exact
+on both sides); attention outputs within max-abs 2e-2 of the oracle's FP64
+result rounded to BF16.  Small cases compare every row; the full-size
+workloads compare sampled rows (first rows, tile and capacity boundaries,
+the last rows, and a seeded random spread) and check properties of all rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+ATOL = 2e-2
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from sparse_attention_10_b200 import build
+    build.build()
+    import sparse_attention_10_b200 as m
+    m.load()
+    return m
+
+
+def to_dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def bf16(a):
+    return to_dev(a).view(torch.bfloat16)
+
+
+def bits_to_f32(a):
+    return (np.asarray(a, dtype=np.uint32) << 16).view(np.float32)
+
+
+def run_prefill(dsa, x, top_k, **kw):
+    q, k = to_dev(x["q_idx"]), to_dev(x["k_idx"])
+    if q.dtype == torch.uint16:
+        q, k = q.view(torch.bfloat16), k.view(torch.bfloat16)
+    ws = torch.empty(dsa.dsa_prefill_workspace_size(q.shape[0], q.shape[1], 0 if q.dtype == torch.uint8 else 1,
+                                                    x["Q"].shape[1], x["Q"].shape[2], top_k),
+                     dtype=torch.uint8, device="cuda")
+    idx, O = dsa.dsa_prefill(q, k, bf16(x["Q"]), bf16(x["K"]), bf16(x["V"]), top_k, workspace=ws, **kw)
+    assert dsa.dsa_sync_status() == 0
+    stats = dsa.dsa_last_stats(ws)
+    return idx.cpu().numpy(), O.view(torch.int16).cpu().numpy().view(np.uint16), stats
+
+
+def small_inputs(L, d, H, D, idx_dtype="fp8", seed=3, lo=-4, hi=4):
+    key = synth.stream_key(seed, 500, L, d)
+    qi = synth.uniform_ints(key, L * d, lo, hi).reshape(L, d)
+    ki = synth.uniform_ints(key, L * d, lo, hi, start=L * d).reshape(L, d)
+    enc = synth.fp8_bytes_of_ints if idx_dtype == "fp8" else synth.bf16_bits_of_ints
+    return {
+        "q_idx": enc(qi), "k_idx": enc(ki), "L": L,
+        "Q": synth.normal_bf16(synth.stream_key(seed, 1, L), L * H * D).reshape(L, H, D),
+        "K": synth.normal_bf16(synth.stream_key(seed, 2, L), L * D).reshape(L, D),
+        "V": synth.normal_bf16(synth.stream_key(seed, 3, L), L * D).reshape(L, D),
+    }
+
+
+def compare(x, idx_dtype, top_k, idx, O, rows=None):
+    ri, ro = oracle.prefill_rows(x, idx_dtype, top_k, rows=rows)
+    sel = slice(None) if rows is None else rows
+    gi = idx[sel]
+    bad = np.nonzero((gi != ri).any(axis=1))[0]
+    assert bad.size == 0, f"indices differ on rows {np.asarray(rows if rows is not None else np.arange(len(ri)))[bad[:10]]}"
+    err = np.abs(bits_to_f32(O[sel]) - bits_to_f32(ro)).max()
+    assert err <= ATOL, f"max-abs error {err}"
+
+
+# ------------------------------------------------------------------ indexer
+
+@pytest.mark.parametrize("idx_dtype,d,Lq,Lk", [
+    ("fp8", 128, 300, 517), ("fp8", 96, 129, 257), ("bf16", 160, 200, 300),
+    ("fp8", 32, 1, 1), ("bf16", 16, 130, 70), ("fp8", 256, 64, 1000), ("bf16", 256, 40, 260),
+])
+def test_indexer_scores_bit_exact(dsa, idx_dtype, d, Lq, Lk):
+    key = synth.stream_key(77, d, Lq, Lk)
+    enc = synth.fp8_bytes_of_ints if idx_dtype == "fp8" else synth.bf16_bits_of_ints
+    q = enc(synth.uniform_ints(key, Lq * d).reshape(Lq, d))
+    k = enc(synth.uniform_ints(key, Lk * d, start=Lq * d).reshape(Lk, d))
+    qt, kt = to_dev(q), to_dev(k)
+    if idx_dtype == "bf16":
+        qt, kt = qt.view(torch.bfloat16), kt.view(torch.bfloat16)
+    got = dsa.dsa_indexer_scores(qt, kt).cpu().numpy()
+    assert dsa.dsa_sync_status() == 0
+    ref = oracle.indexer_scores(q, k, idx_dtype)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_indexer_scores_general_fp8_close(dsa):
+    rng = np.random.default_rng(1)
+    b = rng.integers(0, 256, size=(200, 128), dtype=np.uint8)
+    b = np.where((b & 0x7F) == 0x7F, np.uint8(0x3C), b)
+    c = rng.integers(0, 256, size=(300, 128), dtype=np.uint8)
+    c = np.where((c & 0x7F) == 0x7F, np.uint8(0x3C), c)
+    got = dsa.dsa_indexer_scores(to_dev(b), to_dev(c)).cpu().numpy()
+    ref = oracle.indexer_scores(b, c, "fp8")
+    assert np.allclose(got, ref, rtol=1e-5, atol=1e-5 * np.abs(ref).max())
+
+
+# ------------------------------------------------------------------ prefill, small
+
+@pytest.mark.parametrize("L,top_k", [(1, 16), (5, 16), (129, 64), (700, 256), (2000, 256), (1500, 64)])
+def test_prefill_small_all_rows(dsa, L, top_k):
+    x = small_inputs(L, 128, 4, 64)
+    idx, O, _ = run_prefill(dsa, x, top_k)
+    compare(x, "fp8", top_k, idx, O)
+
+
+def test_prefill_d96_ragged(dsa):
+    x = small_inputs(2333, 96, 16, 128, seed=5)
+    idx, O, _ = run_prefill(dsa, x, 128)
+    compare(x, "fp8", 128, idx, O)
+
+
+def test_prefill_bf16_index(dsa):
+    x = small_inputs(1900, 160, 16, 128, idx_dtype="bf16", seed=6)
+    idx, O, _ = run_prefill(dsa, x, 300)
+    compare(x, "bf16", 300, idx, O)
+
+
+def test_prefill_many_ties(dsa):
+    # Index values in {-1, 0, 1}: scores take few values, so ties cross the k-th place.
+    x = small_inputs(3000, 32, 2, 64, seed=8, lo=-1, hi=1)
+    idx, O, _ = run_prefill(dsa, x, 200)
+    compare(x, "fp8", 200, idx, O)
+
+
+def test_prefill_all_zero_scores(dsa):
+    x = small_inputs(2500, 128, 4, 64, seed=9)
+    x["q_idx"] = np.zeros_like(x["q_idx"])
+    idx, O, stats = run_prefill(dsa, x, 256)
+    for t in (0, 10, 255, 256, 2499):
+        m = min(256, t + 1)
+        assert idx[t, :m].tolist() == list(range(m))
+    compare(x, "fp8", 256, idx, O, rows=np.array([0, 1, 300, 1000, 2499]))
+
+
+def test_prefill_top_k_2048_small(dsa):
+    x = small_inputs(5000, 128, 16, 128, seed=10)
+    idx, O, _ = run_prefill(dsa, x, 2048)
+    rows = np.unique(np.concatenate([np.arange(0, 5000, 97), [2047, 2048, 4095, 4096, 4999]]))
+    compare(x, "fp8", 2048, idx, O, rows=rows)
+
+
+def test_prefill_explicit_scales(dsa):
+    x = small_inputs(900, 128, 4, 64, seed=11)
+    idx, O, _ = run_prefill(dsa, x, 100, idx_scale=0.25, attn_scale=0.05)
+    ri, ro = oracle.prefill_rows(x, "fp8", 100, idx_scale=0.25, attn_scale=0.05)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_prefill_workload_4k_all_rows(dsa):
+    w = synth.WORKLOADS["prefill_4k"]
+    x = synth.prefill_inputs(w)
+    idx, O, stats = run_prefill(dsa, x, w.top_k)
+    compare(x, w.idx_dtype, w.top_k, idx, O)
+
+
+# ------------------------------------------------------------------ prefill, full size
+
+def sampled_rows(L, k, n=48, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, k - 2, k - 1, k, k + 1, 2 * k, 4 * k, L // 2, L - 129, L - 128, L - 2, L - 1]
+    rows = np.concatenate([np.array([r for r in fixed if 0 <= r < L]), rng.integers(0, L, n)])
+    return np.unique(rows).astype(np.int64)
+
+
+def check_index_properties(idx, top_k):
+    t = torch.from_numpy(idx).cuda()
+    L = t.shape[0]
+    m = torch.clamp(torch.arange(L, device="cuda") + 1, max=top_k)
+    col = torch.arange(top_k, device="cuda")[None, :]
+    valid = col < m[:, None]
+    assert bool(((t >= 0) == valid).all()), "-1 padding in the wrong place"
+    assert bool((t[valid] <= torch.arange(L, device="cuda")[:, None].expand_as(t)[valid]).all()), "non-causal index"
+    s, _ = torch.sort(torch.where(valid, t, torch.full_like(t, -1)), dim=1)
+    dup = (s[:, 1:] == s[:, :-1]) & (s[:, 1:] >= 0)
+    assert not bool(dup.any()), "duplicate index in a row"
+
+
+@pytest.mark.parametrize("name", ["prefill_32k", "prefill_64k", "prefill_128k"])
+def test_prefill_full_workloads_sampled(dsa, name):
+    w = synth.WORKLOADS[name]
+    x = synth.prefill_inputs(w)
+    idx, O, stats = run_prefill(dsa, x, w.top_k)
+    check_index_properties(idx, w.top_k)
+    rows = sampled_rows(w.L, w.top_k)
+    compare(x, w.idx_dtype, w.top_k, idx, O, rows=rows)
+    assert stats["fallback_rows"] < w.L // 100, stats
+
+
+# ------------------------------------------------------------------ decode
+
+def run_decode(dsa, xd, top_k):
+    t = {k: to_dev(xd[k]) for k in ("k_idx", "K", "V", "q_idx", "Q", "seq_start")}
+    O, idx = dsa.dsa_decode(t["k_idx"], t["K"].view(torch.bfloat16), t["V"].view(torch.bfloat16),
+                            t["seq_start"], t["q_idx"], t["Q"].view(torch.bfloat16), top_k,
+                            int(xd["lengths"].max()))
+    assert dsa.dsa_sync_status() == 0
+    return idx.cpu().numpy(), O.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def test_decode_small_ragged(dsa):
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([1, 2, 100, 2047, 2048, 2049, 4097, 9000, 70000], dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    idx, O = run_decode(dsa, xd, w.top_k)
+    ri, ro = oracle.decode(xd, w.idx_dtype, w.top_k)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_decode_small_top_k(dsa):
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([3, 50, 777], dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    idx, O = run_decode(dsa, xd, 40)
+    ri, ro = oracle.decode(xd, w.idx_dtype, 40)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_decode_full_workload(dsa):
+    w = synth.WORKLOADS["decode_64x128k"]
+    xd = synth.decode_inputs(w)
+    idx, O = run_decode(dsa, xd, w.top_k)
+    ri, ro = oracle.decode(xd, w.idx_dtype, w.top_k)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives(dsa):
+    assert dsa.dsa_sync_status() == 0
+    dsa.dsa_debug_wait_timeout(1_000_000)   # 1 ms, nothing completes the barrier
+    assert dsa.dsa_sync_status() == 5       # DSA_ERR_TIMEOUT, read and cleared
+    assert dsa.dsa_sync_status() == 0
+    x = small_inputs(300, 128, 4, 64, seed=12)
+    idx, O, _ = run_prefill(dsa, x, 32)
+    compare(x, "fp8", 32, idx, O)
