@@ -1,0 +1,438 @@
+"""Benchmark of the DSA hot path on B200.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one dsa_prefill of the 128K workload (L = 131072, index dim 160 in
+BF16, H = 16, D = 128, top_k = 2048): indexer sample + threshold + causal
+indexer with fused filter + exact select + gathered attention.  `value` is
+whole-job prefill queries/s (each rank runs its own sequence: weak scaling,
+no data-path collective).  The decode rows of the path (64 sequences with
+cached lengths in [65536, 131072], top_k 2048) are timed in their own K-step
+loop and reported under "decode".  Inputs are synthetic and seeded; each
+step's working set (~9 GB) is far larger than the 126 MB L2.
+
+--impl reference times the CPU oracle (the plain restatement the tests check
+against) on a bounded sample of query rows per step, on the host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "DSA prefill queries/s @128K (indexer TFLOP/s, gather GB/s); decode tok/s"
+PREFILL = "prefill_128k"
+DECODE = "decode_64x128k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample time")
+    return ap.parse_args()
+
+
+def rank_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        p.update({k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in m})
+        p["source"] = "measured"
+    except (OSError, ValueError, KeyError):
+        pass
+    return p
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU every 100 ms (NVML)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.1)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- work accounting
+
+def prefill_work(w):
+    L, k, d, D, H = w.L, w.top_k, w.d_idx, w.D, w.H
+    pairs = L * (L + 1) // 2                      # causal pairs, diagonal included
+    kept = sum(min(t + 1, k) for t in range(min(L, k))) + max(0, L - k) * k
+    return {
+        "indexer_flops": 2.0 * d * pairs,
+        "gather_bytes": float(kept) * 2 * D * 2,  # one K row + one V row per kept key
+        "attn_flops": 4.0 * H * D * kept,
+        "attn_bytes": float(kept) * 2 * D * 2 + 2.0 * L * H * D * 2 + 4.0 * L * k,
+        "kept": kept,
+    }
+
+
+def decode_work(w, lengths):
+    total = int(lengths.sum())
+    kept = int(np.minimum(lengths, w.top_k).sum())
+    esize = 1 if w.idx_dtype == "fp8" else 2
+    return {
+        "scan_bytes": float(total) * w.d_idx * esize + total * 4.0,   # read index rows, write scores
+        "gather_bytes": float(kept) * 2 * w.D * 2,
+        "total_rows": total,
+    }
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def cpu_oracle_sample(w, host, target_s, seed=0, rows=None):
+    """Time the oracle on evenly spread query rows; returns (queries/s, rows, seconds, threads)."""
+    import oracle
+    threads = oracle.max_threads()
+    if rows is None:
+        # calibrate on a small batch, then size the sample to ~target_s
+        probe = np.linspace(0, w.L - 1, max(4, threads), dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=probe)
+        dt = time.perf_counter() - t0
+        n = int(max(len(probe), min(w.L, len(probe) * target_s / max(dt, 1e-3))))
+        rng = np.random.default_rng(seed)
+        rows = np.sort(rng.choice(w.L, size=n, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
+    dt = time.perf_counter() - t0
+    return len(rows) / dt, len(rows), dt, threads
+
+
+def host_copy(x):
+    import torch
+    out = {}
+    for k, v in x.items():
+        if isinstance(v, torch.Tensor):
+            t = v.cpu()
+            if t.dtype == torch.bfloat16:
+                t = t.view(torch.int16)
+            out[k] = t.numpy().view(np.uint16) if t.dtype == torch.int16 else t.numpy()
+        else:
+            out[k] = v
+    return out
+
+
+def run_reference(args):
+    import synth
+    rank, world, _ = rank_info()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[PREFILL]
+    host = synth.prefill_inputs(w)
+    per_step = max(2.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    # size one step's sample from a calibration run (untimed)
+    import oracle
+    threads = oracle.max_threads()
+    probe = np.linspace(0, w.L - 1, max(4, threads), dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=probe)
+    n = int(max(len(probe), len(probe) * per_step / max(time.perf_counter() - t0, 1e-3)))
+    rng = np.random.default_rng(1)
+    times = []
+    for step in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(w.L, size=n, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
+        if step >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = n * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{PREFILL}: L=131072 causal, q_idx/k_idx [L,160] bf16 ints in [-4,4], "
+                               f"Q [L,16,128], K/V [L,128] bf16 N(0,1), top_k=2048",
+                   "sample_rows_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} random query rows of {PREFILL} per step (full work of each row)"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def main():
+    args = parse()
+    rank, world, local = rank_info()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    import torch.distributed as dist
+
+    import synth
+    import sparse_attention_10_b200 as dsa
+    from sparse_attention_10_b200 import build as dsa_build
+
+    dsa_build.build()
+    dsa.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = synth.WORKLOADS[PREFILL]
+    seed = synth.SEED + rank              # every rank runs its own sequence
+    x = synth.prefill_inputs_torch(w, seed=seed, device=dev)
+    q, k = x["q_idx"], x["k_idx"]
+    Q, K, V = x["Q"], x["K"], x["V"]
+    idt = dsa.IDX_BF16 if w.idx_dtype == "bf16" else dsa.IDX_FP8_E4M3
+    ws = torch.empty(dsa.dsa_prefill_workspace_size(w.L, w.d_idx, idt, w.H, w.D, w.top_k),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty((w.L, w.top_k), dtype=torch.int32, device=dev)
+    O = torch.empty((w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dsa.dsa_prefill(q, k, Q, K, V, w.top_k, indices=idx, O=O, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if dsa.dsa_sync_status(stream) != 0:
+        raise RuntimeError("device-side error during warm-up")
+    stats = dsa.dsa_last_stats(ws)
+
+    # --- timed region: K prefill steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    if dsa.dsa_sync_status(stream) != 0:
+        raise RuntimeError("device-side error in the timed region")
+    value = world * w.L * args.steps / (ms / 1000.0)
+
+    # --- per-stage times: the same K steps again with stage events on the stream
+    dsa.dsa_stage_timing(True)
+    for _ in range(args.steps):
+        step()
+    torch.cuda.synchronize()
+    dsa.dsa_stage_timing(False)
+    stages = dsa.dsa_stage_times()
+    launches_per_step = sum(v[1] for v in stages.values()) / args.steps
+    work = prefill_work(w)
+    pk = peaks()
+    st_ms = {k_: v[0] / args.steps for k_, v in stages.items() if v[1] > 0}
+    idx_ms = st_ms.get("indexer_filter", float("nan"))
+    att_ms = st_ms.get("attention", float("nan"))
+    indexer_tflops = work["indexer_flops"] / (idx_ms / 1000.0) / 1e12
+    gather_gbs = work["gather_bytes"] / (att_ms / 1000.0) / 1e9
+    dominant = max(("indexer_filter", "attention", "select", "indexer_sample", "threshold"),
+                   key=lambda s: st_ms.get(s, 0.0))
+    if dominant.startswith("indexer"):
+        flops = work["indexer_flops"] if dominant == "indexer_filter" else float("nan")
+        ach = flops / (st_ms[dominant] / 1000.0) / 1e12
+        roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"], "traffic": None}
+    else:
+        ach = work["attn_bytes"] / (st_ms["attention"] / 1000.0) / 1e9 if dominant == "attention" else float("nan")
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": None}
+    roof["peak_source"] = pk["source"]
+
+    # --- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory(); hk = k.cpu().pin_memory()
+        hQ = Q.cpu().pin_memory(); hK = K.cpu().pin_memory(); hV = V.cpu().pin_memory()
+        hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        dq, dk, dQ, dK, dV = (torch.empty_like(t, device=dev) for t in (hq, hk, hQ, hK, hV))
+
+        def e2e_step():
+            for d_, h_ in ((dq, hq), (dk, hk), (dQ, hQ), (dK, hK), (dV, hV)):
+                d_.copy_(h_, non_blocking=True)
+            dsa.dsa_prefill(dq, dk, dQ, dK, dV, w.top_k, indices=idx, O=O, workspace=ws, stream=stream)
+            hidx.copy_(idx, non_blocking=True)
+            hO.copy_(O, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, args.steps // 2)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hQ, hK, hV))
+        d2h = idx.numel() * 4 + O.numel() * 2
+        e2e = {"value": world * w.L * n_e2e / (ems / 1000.0), "unit": "queries/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": ems / n_e2e}
+        del dq, dk, dQ, dK, dV, hq, hk, hQ, hK, hV, hidx, hO
+
+    # --- decode rows of the path
+    decode = None
+    if not args.no_decode:
+        wd = synth.WORKLOADS[DECODE]
+        del ws
+        torch.cuda.empty_cache()
+        xd = synth.decode_inputs_torch(wd, seed=seed, device=dev)
+        lengths = xd["lengths"]
+        wsd = torch.empty(dsa.dsa_decode_workspace_size(wd.B, int(lengths.sum()), wd.d_idx, 0, wd.H, wd.D,
+                                                         wd.top_k), dtype=torch.uint8, device=dev)
+        Od = torch.empty((wd.B, wd.H, wd.D), dtype=torch.bfloat16, device=dev)
+        idd = torch.empty((wd.B, wd.top_k), dtype=torch.int32, device=dev)
+
+        def dstep():
+            dsa.dsa_decode(xd["k_idx"], xd["K"], xd["V"], xd["seq_start"], xd["q_idx"], xd["Q"], wd.top_k,
+                           int(lengths.max()), O=Od, indices=idd, workspace=wsd, stream=stream)
+
+        for _ in range(args.warmup):
+            dstep()
+        torch.cuda.synchronize()
+        nd = max(args.steps, 20)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(nd):
+            dstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(e0.elapsed_time(e1))
+        dsa.dsa_stage_timing(True)
+        for _ in range(nd):
+            dstep()
+        torch.cuda.synchronize()
+        dsa.dsa_stage_timing(False)
+        dst = {k_: v[0] / nd for k_, v in dsa.dsa_stage_times().items() if v[1] > 0}
+        dw = decode_work(wd, lengths)
+        scan_ms = dst.get("decode_scan_select", float("nan"))
+        decode = {"metric": "decode tok/s", "value": world * wd.B * nd / (dms / 1000.0), "unit": "tok/s",
+                  "ms_per_step": dms / nd, "workload": f"{DECODE}: B=64, cached lengths U[65536,131072] "
+                  f"(sum {dw['total_rows']}), k_idx fp8 d=128, H=16, D=128, top_k=2048",
+                  "stage_ms": dst,
+                  "scan_select_gbs": dw["scan_bytes"] / (scan_ms / 1000.0) / 1e9,
+                  "scan_select_frac_hbm": dw["scan_bytes"] / (scan_ms / 1000.0) / 1e9 / pk["hbm_gbs"]}
+        if dsa.dsa_sync_status(stream) != 0:
+            raise RuntimeError("device-side error in decode")
+
+    # --- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_copy(x)
+        qps, n, dt, thr = cpu_oracle_sample(w, host, args.cpu_seconds)
+        cpu = {"value": qps, "unit": "queries/s", "cores": thr, "kind": "oracle",
+               "sample": f"{n} random query rows of {PREFILL} (full work of each row: indexer over "
+                         f"t+1 keys, top-2048, attention), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{PREFILL}: L=131072 causal, q_idx/k_idx [L,160] bf16 ints in [-4,4], "
+                                   f"Q [L,16,128], K/V [L,128] bf16 N(0,1), top_k=2048",
+                       "parallelism": f"{world} independent sequences (one per GPU)",
+                       "l2": "inputs larger than L2 (~9 GB touched per step vs 126 MB L2)"},
+            "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs,
+            "stage_ms": st_ms, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clocks.summary(),
+            "decode": decode, "select_stats": stats,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -160,6 +160,21 @@ dsa_status dsa_sync_status(void* stream);
 dsa_status dsa_last_stats(const void* workspace, int64_t out[4], void* stream);
 
 /*
+ * Stage timing (diagnostic).  While enabled (per process), dsa_prefill and
+ * dsa_decode record a CUDA event before and after each of their stages on
+ * the call's stream.  dsa_stage_times synchronises those events, writes the
+ * summed time in milliseconds and the number of kernel launches of each stage
+ * into ms[i] / launches[i] for i < n (n <= DSA_NUM_STAGES), and resets them.
+ * Stages: 0 indexer sample, 1 threshold, 2 indexer filter, 3 select +
+ * fallback, 4 attention, 5 decode scan, 6 decode select, 7 decode attention
+ * + combine (stage 5 covers the whole decode scan and select; stage 6 is
+ * unused).  Events are created on demand and kept for reuse.
+ */
+#define DSA_NUM_STAGES 8
+dsa_status dsa_stage_timing(int enable);
+dsa_status dsa_stage_times(double* ms, int64_t* launches, int n);
+
+/*
  * dsa_debug_wait_timeout — runs one tiny kernel whose only work is a
  * bounded wait on a shared-memory barrier that nothing completes, with a
  * limit of `limit_ns` nanoseconds.  The kernel records DSA_ERR_TIMEOUT in the

@@ -18,7 +18,7 @@ __all__ = [
     "DsaError", "load", "dsa_version", "dsa_status_string", "dsa_indexer_scores",
     "dsa_prefill_workspace_size", "dsa_prefill", "dsa_decode_workspace_size", "dsa_decode",
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "IDX_FP8_E4M3", "IDX_BF16",
-    "LIB_PATH",
+    "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
         "dsa_sync_status": ([P], I),
         "dsa_last_stats": ([P, ctypes.POINTER(ctypes.c_int64), P], I),
         "dsa_debug_wait_timeout": ([ctypes.c_uint64, P], I),
+        "dsa_stage_timing": ([I], I),
+        "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -197,6 +199,23 @@ def dsa_last_stats(workspace: torch.Tensor, stream=None) -> dict:
 
 def dsa_debug_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(load().dsa_debug_wait_timeout(int(limit_ns), _stream(stream)), "dsa_debug_wait_timeout")
+
+
+STAGES = ["indexer_sample", "threshold", "indexer_filter", "select", "attention",
+          "decode_scan_select", "unused", "decode_attention"]
+
+
+def dsa_stage_timing(enable: bool) -> None:
+    _check(load().dsa_stage_timing(1 if enable else 0), "dsa_stage_timing")
+
+
+def dsa_stage_times() -> dict:
+    """{stage: (milliseconds, kernel launches)} summed since the last read (then reset)."""
+    n = len(STAGES)
+    ms = (ctypes.c_double * n)()
+    ln = (ctypes.c_int64 * n)()
+    _check(load().dsa_stage_times(ms, ln, n), "dsa_stage_times")
+    return {STAGES[i]: (ms[i], int(ln[i])) for i in range(n)}
 
 
 def default_index_scale(d: int) -> float:

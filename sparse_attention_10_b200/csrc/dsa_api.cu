@@ -11,6 +11,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -106,6 +108,54 @@ DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k) {
   p.total = o;
   return p;
 }
+
+// ---- stage timing (diagnostic) -------------------------------------------------------
+
+struct StageRec {
+  cudaEvent_t a, b;
+  int stage, launches;
+};
+bool g_timing = false;
+std::mutex g_timing_mu;
+std::vector<StageRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+double g_ms[DSA_NUM_STAGES];
+int64_t g_launches[DSA_NUM_STAGES];
+
+cudaEvent_t pooled_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Records an event on `s` at construction and at destruction (when enabled).
+class StageScope {
+ public:
+  StageScope(int stage, int launches, cudaStream_t s) : stage_(stage), launches_(launches), s_(s) {
+    if (!g_timing) return;
+    std::lock_guard<std::mutex> g(g_timing_mu);
+    a_ = pooled_event();
+    if (a_) cudaEventRecord(a_, s_);
+  }
+  ~StageScope() {
+    if (!g_timing || !a_) return;
+    std::lock_guard<std::mutex> g(g_timing_mu);
+    cudaEvent_t b = pooled_event();
+    if (!b) return;
+    cudaEventRecord(b, s_);
+    g_recs.push_back({a_, b, stage_, launches_});
+  }
+
+ private:
+  int stage_, launches_;
+  cudaStream_t s_;
+  cudaEvent_t a_ = nullptr;
+};
 
 __global__ void wait_timeout_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
@@ -225,21 +275,27 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   a.scale = iscale;
   a.limit_ns = wait_limit_ns();
   if (L > plan.cap_all) {
+    StageScope scope(0, 1, s);
     a.mode = kModeSample;
     a.samp = samp;
     a.samp_ld = plan.samp_ld;
     a.cap = plan.cap_all;
     if ((st = launch_indexer(a, s)) != DSA_OK) return st;
   }
-  if ((st = launch_tau_select(samp, plan.samp_ld, L, plan.cap_all, plan.target, iscale, tau, s)) !=
-      DSA_OK)
-    return st;
+  {
+    StageScope scope(1, 1, s);
+    st = launch_tau_select(samp, plan.samp_ld, L, plan.cap_all, plan.target, iscale, tau, s);
+    if (st != DSA_OK) return st;
+  }
   a.mode = kModeFilter;
   a.tau = tau;
   a.cand = cand;
   a.cand_n = cand_n;
   a.cap = plan.cap_half;
-  if ((st = launch_indexer(a, s)) != DSA_OK) return st;
+  {
+    StageScope scope(2, 1, s);
+    if ((st = launch_indexer(a, s)) != DSA_OK) return st;
+  }
 
   SelectLaunch sl{};
   sl.L = L;
@@ -257,7 +313,10 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   sl.scale = iscale;
   sl.fb_scratch = fb_scratch;
   sl.fb_ctas = plan.fb_ctas;
-  if ((st = launch_select(sl, s)) != DSA_OK) return st;
+  {
+    StageScope scope(3, 2, s);
+    if ((st = launch_select(sl, s)) != DSA_OK) return st;
+  }
 
   AttnLaunch at{};
   at.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -273,6 +332,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   at.seq_start = nullptr;
   at.nsplit = 1;
   at.O = static_cast<__nv_bfloat16*>(O);
+  StageScope scope(4, 1, s);
   return launch_attention(at, s);
 }
 
@@ -327,7 +387,10 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
   dl.indices = idx;
   dl.keys = reinterpret_cast<unsigned long long*>(ws + plan.off_keys);
   dl.invalid = reinterpret_cast<int*>(ws + plan.off_counters) + 8;
-  if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
+  {
+    StageScope scope(5, 3, s);  // validate + scan + select (timed together)
+    if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
+  }
 
   AttnLaunch at{};
   at.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -345,6 +408,7 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
   at.O = static_cast<__nv_bfloat16*>(O);
   at.part = reinterpret_cast<float*>(ws + plan.off_part);
   at.invalid = dl.invalid;
+  StageScope scope(7, 2, s);
   return launch_attention(at, s);
 }
 
@@ -365,6 +429,37 @@ dsa_status dsa_last_stats(const void* workspace, int64_t out[4], void* stream) {
     return DSA_ERR_CUDA;
   for (int i = 0; i < 4; ++i) out[i] = c[i];
   return DSA_OK;
+}
+
+dsa_status dsa_stage_timing(int enable) {
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  g_timing = enable != 0;
+  return DSA_OK;
+}
+
+dsa_status dsa_stage_times(double* ms, int64_t* launches, int n) {
+  if (n < 0 || n > DSA_NUM_STAGES) return DSA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> g(g_timing_mu);
+  dsa_status st = DSA_OK;
+  for (const StageRec& r : g_recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = DSA_ERR_CUDA;
+    g_ms[r.stage] += t;
+    g_launches[r.stage] += r.launches;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  for (int i = 0; i < n; ++i) {
+    if (ms) ms[i] = g_ms[i];
+    if (launches) launches[i] = g_launches[i];
+  }
+  for (int i = 0; i < DSA_NUM_STAGES; ++i) {
+    g_ms[i] = 0.0;
+    g_launches[i] = 0;
+  }
+  return st;
 }
 
 dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
 from typing import Optional
 
 import numpy as np
@@ -107,25 +108,40 @@ def bf16_bits_of_f32(x: np.ndarray) -> np.ndarray:
         return ((u + bias) >> np.uint32(16)).astype(np.uint16)
 
 
-def normal_bf16(key: np.uint64, n: int, chunk: int = 1 << 24) -> np.ndarray:
-    """n N(0,1) values as BF16 bit patterns (Box-Muller, both outputs of a pair)."""
+def normal_bf16(key: np.uint64, n: int, chunk: int = 1 << 22, workers: int = 0) -> np.ndarray:
+    """n N(0,1) values as BF16 bit patterns (Box-Muller, both outputs of a pair).
+
+    Chunks are independent slices of the counter stream, so the result does not
+    depend on ``workers`` (threads; 0 = one per CPU, capped at 32).
+    """
     out = np.empty(n, dtype=np.uint16)
     npairs = (n + 1) // 2
-    two_pi = 2.0 * math.pi
-    for p0 in range(0, npairs, chunk):
-        m = min(chunk, npairs - p0)
-        z = draws(key, p0, m)
-        u1 = ((z >> np.uint64(32)).astype(np.float64) + 0.5) * (1.0 / 4294967296.0)
-        u2 = ((z & np.uint64(0xFFFFFFFF)).astype(np.float64) + 0.5) * (1.0 / 4294967296.0)
-        r = np.sqrt(-2.0 * np.log(u1))
-        th = two_pi * u2
-        pair = np.empty(2 * m, dtype=np.float32)
-        pair[0::2] = r * np.cos(th)
-        pair[1::2] = r * np.sin(th)
-        lo = 2 * p0
-        hi = min(n, lo + 2 * m)
-        out[lo:hi] = bf16_bits_of_f32(pair[: hi - lo])
+    starts = list(range(0, npairs, chunk))
+    if workers == 0:
+        workers = min(32, os.cpu_count() or 1)
+    if workers > 1 and len(starts) > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(lambda p0: _normal_chunk(key, p0, min(chunk, npairs - p0), n, out), starts))
+    else:
+        for p0 in starts:
+            _normal_chunk(key, p0, min(chunk, npairs - p0), n, out)
     return out
+
+
+def _normal_chunk(key, p0, m, n, out):
+    """Pairs p0 .. p0+m-1 of the stream into out[2*p0 : 2*(p0+m)] (clipped to n)."""
+    z = draws(key, p0, m)
+    u1 = ((z >> np.uint64(32)).astype(np.float64) + 0.5) * (1.0 / 4294967296.0)
+    u2 = ((z & np.uint64(0xFFFFFFFF)).astype(np.float64) + 0.5) * (1.0 / 4294967296.0)
+    r = np.sqrt(-2.0 * np.log(u1))
+    th = (2.0 * math.pi) * u2
+    pair = np.empty(2 * m, dtype=np.float32)
+    pair[0::2] = r * np.cos(th)
+    pair[1::2] = r * np.sin(th)
+    lo = 2 * p0
+    hi = min(n, lo + 2 * m)
+    out[lo:hi] = bf16_bits_of_f32(pair[: hi - lo])
 
 
 @dataclasses.dataclass(frozen=True)
@@ -245,3 +261,106 @@ def decode_inputs(w: Workload, seed: int = SEED, lengths: Optional[np.ndarray] =
         out["K"] = _prefix_normal(seed, w.cid, _T_K, total * w.D).reshape(total, w.D)
         out["V"] = _prefix_normal(seed, w.cid, _T_V, total * w.D).reshape(total, w.D)
     return out
+
+
+# ---------------------------------------------------------------------------
+# The same generators written with torch integer/float ops, so large inputs can
+# be drawn directly on a device.  Definitions match the numpy ones above draw
+# for draw (64-bit wrapping arithmetic in int64, logical shifts emulated).
+
+def _to_i64(u: int) -> int:
+    u &= 0xFFFFFFFFFFFFFFFF
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+_M1_I, _M2_I, _G_I = _to_i64(0xBF58476D1CE4E5B9), _to_i64(0x94D049BB133111EB), _to_i64(0x9E3779B97F4A7C15)
+
+
+def _srl(x, s: int):
+    return (x >> s) & ((1 << (64 - s)) - 1)
+
+
+def draws_torch(key, start: int, n: int, device):
+    import torch
+    i = torch.arange(start + 1, start + n + 1, dtype=torch.int64, device=device)
+    z = i * _G_I + _to_i64(int(key))
+    z = (z ^ _srl(z, 30)) * _M1_I
+    z = (z ^ _srl(z, 27)) * _M2_I
+    return z ^ _srl(z, 31)
+
+
+def uniform_ints_torch(key, n: int, lo: int = -4, hi: int = 4, device="cuda", chunk: int = 1 << 26):
+    import torch
+    out = torch.empty(n, dtype=torch.int8, device=device)
+    for s in range(0, n, chunk):
+        m = min(chunk, n - s)
+        top = _srl(draws_torch(key, s, m, device), 32)
+        out[s:s + m] = ((top * (hi - lo + 1)) >> 32).to(torch.int8) + lo
+    return out
+
+
+def normal_bf16_torch(key, n: int, device="cuda", chunk: int = 1 << 25):
+    """N(0,1) as a torch.bfloat16 tensor on `device` (same draws as normal_bf16)."""
+    import torch
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    npairs = (n + 1) // 2
+    for p0 in range(0, npairs, chunk):
+        m = min(chunk, npairs - p0)
+        z = draws_torch(key, p0, m, device)
+        u1 = (_srl(z, 32).to(torch.float64) + 0.5) * (1.0 / 4294967296.0)
+        u2 = ((z & 0xFFFFFFFF).to(torch.float64) + 0.5) * (1.0 / 4294967296.0)
+        r = torch.sqrt(-2.0 * torch.log(u1))
+        th = (2.0 * math.pi) * u2
+        pair = torch.stack([(r * torch.cos(th)).to(torch.float32),
+                            (r * torch.sin(th)).to(torch.float32)], dim=1).reshape(-1)
+        lo = 2 * p0
+        hi = min(n, lo + 2 * m)
+        out[lo:hi] = pair[: hi - lo].to(torch.bfloat16)
+    return out
+
+
+def _encode_ints_torch(v, idx_dtype: str):
+    import torch
+    if idx_dtype == "fp8":
+        return v.to(torch.float8_e4m3fn).view(torch.uint8)
+    return v.to(torch.bfloat16)
+
+
+def prefill_inputs_torch(w: Workload, seed: int = SEED, device="cuda") -> dict:
+    """prefill_inputs drawn on a device: uint8 / bfloat16 torch tensors."""
+    import torch
+    L = w.L
+    qi = uniform_ints_torch(stream_key(seed, w.cid, _T_QIDX), L * w.d_idx, device=device).view(L, w.d_idx)
+    ki = uniform_ints_torch(stream_key(seed, w.cid, _T_KIDX), L * w.d_idx, device=device).view(L, w.d_idx)
+    if w.local_boost:
+        nblk = (L + 127) // 128
+        u = uniform_ints_torch(stream_key(seed, w.cid, _T_BOOST), nblk * 32, device=device).view(nblk, 32)
+        blk = torch.arange(L, device=device) // 128
+        qi[:, :32] = u[blk]
+        ki[:, :32] = u[blk]
+    return {
+        "q_idx": _encode_ints_torch(qi, w.idx_dtype), "k_idx": _encode_ints_torch(ki, w.idx_dtype), "L": L,
+        "Q": normal_bf16_torch(stream_key(seed, w.cid, _T_Q), L * w.H * w.D, device).view(L, w.H, w.D),
+        "K": normal_bf16_torch(stream_key(seed, w.cid, _T_K), L * w.D, device).view(L, w.D),
+        "V": normal_bf16_torch(stream_key(seed, w.cid, _T_V), L * w.D, device).view(L, w.D),
+    }
+
+
+def decode_inputs_torch(w: Workload, seed: int = SEED, device="cuda") -> dict:
+    """decode_inputs drawn on a device (drawn lengths)."""
+    import torch
+    lengths = decode_lengths(w, seed)
+    B = lengths.shape[0]
+    seq_start = np.zeros(B + 1, dtype=np.int64)
+    seq_start[1:] = np.cumsum(lengths)
+    total = int(seq_start[-1])
+    ki = uniform_ints_torch(stream_key(seed, w.cid, _T_KIDX), total * w.d_idx, device=device)
+    qi = uniform_ints_torch(stream_key(seed, w.cid, _T_QIDX), B * w.d_idx, device=device)
+    return {
+        "k_idx": _encode_ints_torch(ki, w.idx_dtype).view(total, w.d_idx),
+        "q_idx": _encode_ints_torch(qi, w.idx_dtype).view(B, w.d_idx),
+        "seq_start": torch.from_numpy(seq_start).to(device), "lengths": lengths, "B": B,
+        "Q": normal_bf16_torch(stream_key(seed, w.cid, _T_Q), B * w.H * w.D, device).view(B, w.H, w.D),
+        "K": normal_bf16_torch(stream_key(seed, w.cid, _T_K), total * w.D, device).view(total, w.D),
+        "V": normal_bf16_torch(stream_key(seed, w.cid, _T_V), total * w.D, device).view(total, w.D),
+    }

@@ -189,10 +189,23 @@ def check_index_properties(idx, top_k):
     assert not bool(dup.any()), "duplicate index in a row"
 
 
+def host_copy(x):
+    out = {}
+    for k, v in x.items():
+        if isinstance(v, torch.Tensor):
+            t = v.cpu()
+            if t.dtype == torch.bfloat16:
+                t = t.view(torch.int16)
+            out[k] = t.numpy().view(np.uint16) if t.dtype == torch.int16 else t.numpy()
+        else:
+            out[k] = v
+    return out
+
+
 @pytest.mark.parametrize("name", ["prefill_32k", "prefill_64k", "prefill_128k"])
 def test_prefill_full_workloads_sampled(dsa, name):
     w = synth.WORKLOADS[name]
-    x = synth.prefill_inputs(w)
+    x = host_copy(synth.prefill_inputs_torch(w, device="cuda"))
     idx, O, stats = run_prefill(dsa, x, w.top_k)
     check_index_properties(idx, w.top_k)
     rows = sampled_rows(w.L, w.top_k)
@@ -233,11 +246,21 @@ def test_decode_small_top_k(dsa):
 
 def test_decode_full_workload(dsa):
     w = synth.WORKLOADS["decode_64x128k"]
-    xd = synth.decode_inputs(w)
+    xd = host_copy(synth.decode_inputs_torch(w, device="cuda"))
     idx, O = run_decode(dsa, xd, w.top_k)
     ri, ro = oracle.decode(xd, w.idx_dtype, w.top_k)
     assert np.array_equal(idx, ri)
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_device_generator_matches_numpy_definition():
+    k = synth.stream_key(5, 6)
+    a = synth.normal_bf16(k, 3_000_001)
+    b = synth.normal_bf16_torch(k, 3_000_001, device="cuda").view(torch.int16).cpu().numpy().view(np.uint16)
+    assert (a == b).mean() > 0.999999
+    a = synth.uniform_ints(k, 1_000_000)
+    b = synth.uniform_ints_torch(k, 1_000_000, device="cuda").cpu().numpy()
+    assert np.array_equal(a, b)
 
 
 # ------------------------------------------------------------------ failure detection
