@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample time")
+    ap.add_argument("--workload", default=PREFILL,
+                    choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k"],
+                    help="prefill workload of a step (smaller ones for profiling)")
     return ap.parse_args()
 
 
@@ -152,22 +155,22 @@ def decode_work(w, lengths):
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
-def cpu_oracle_sample(w, host, target_s, seed=0, rows=None):
-    """Time the oracle on evenly spread query rows; returns (queries/s, rows, seconds, threads)."""
+def cpu_oracle_sample(w, host, target_s, seed=0):
+    """Time the oracle on random query rows of the workload, growing the sample
+    until one run takes at least half of target_s; returns (queries/s, rows,
+    seconds, threads) of that last run."""
     import oracle
     threads = oracle.max_threads()
-    if rows is None:
-        # calibrate on a small batch, then size the sample to ~target_s
-        probe = np.linspace(0, w.L - 1, max(4, threads), dtype=np.int64)
+    rng = np.random.default_rng(seed)
+    n = max(4, 2 * threads)
+    for _ in range(5):
+        rows = np.sort(rng.choice(w.L, size=min(n, w.L), replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=probe)
+        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
         dt = time.perf_counter() - t0
-        n = int(max(len(probe), min(w.L, len(probe) * target_s / max(dt, 1e-3))))
-        rng = np.random.default_rng(seed)
-        rows = np.sort(rng.choice(w.L, size=n, replace=False)).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
-    dt = time.perf_counter() - t0
+        if dt >= 0.5 * target_s or len(rows) == w.L:
+            break
+        n = int(min(w.L, len(rows) * 0.9 * target_s / max(dt, 1e-3)))
     return len(rows) / dt, len(rows), dt, threads
 
 
@@ -259,7 +262,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    w = synth.WORKLOADS[PREFILL]
+    w = synth.WORKLOADS[args.workload]
     seed = synth.SEED + rank              # every rank runs its own sequence
     x = synth.prefill_inputs_torch(w, seed=seed, device=dev)
     q, k = x["q_idx"], x["k_idx"]
@@ -412,16 +415,18 @@ def main():
         host = host_copy(x)
         qps, n, dt, thr = cpu_oracle_sample(w, host, args.cpu_seconds)
         cpu = {"value": qps, "unit": "queries/s", "cores": thr, "kind": "oracle",
-               "sample": f"{n} random query rows of {PREFILL} (full work of each row: indexer over "
-                         f"t+1 keys, top-2048, attention), {dt:.1f} s"}
+               "sample": f"{n} random query rows of {w.name} (full work of each row: indexer over "
+                         f"t+1 keys, top-{w.top_k}, attention), {dt:.1f} s"}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{PREFILL}: L=131072 causal, q_idx/k_idx [L,160] bf16 ints in [-4,4], "
-                                   f"Q [L,16,128], K/V [L,128] bf16 N(0,1), top_k=2048",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if w.idx_dtype == "bf16" else "fp8 indexer / bf16 attention", "data": "synthetic",
+            "config": {"workload": f"{w.name}: L={w.L} causal, q_idx/k_idx [L,{w.d_idx}] {w.idx_dtype} ints "
+                                   f"in [-4,4]{' with local boost' if w.local_boost else ''}, "
+                                   f"Q [L,{w.H},{w.D}], K/V [L,{w.D}] bf16 N(0,1), top_k={w.top_k}",
                        "parallelism": f"{world} independent sequences (one per GPU)",
                        "l2": "inputs larger than L2 (~9 GB touched per step vs 126 MB L2)"},
             "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs,

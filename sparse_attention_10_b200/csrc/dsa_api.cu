@@ -303,6 +303,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   sl.cap = plan.cap_half;
   sl.cand = cand;
   sl.cand_n = cand_n;
+  sl.tau = tau;
   sl.indices = indices;
   sl.fb_rows = fb_rows;
   sl.counters = counters;

@@ -444,7 +444,9 @@ __global__ void __launch_bounds__(256) tau_kernel(const uint16_t* samp, int samp
     float a = __uint_as_float(static_cast<uint32_t>((b1 << 8) | b2) << 16);
     const float sigma = __fmul_rn(a, scale);
     if (!(a > 0.0f) || !(sigma > 0.0f)) {
-      tau[t] = -INFINITY;
+      // The sampled rank falls among ReLU zeros: keep every positive score
+      // (smallest positive threshold) and let the select add zeros by index.
+      tau[t] = __uint_as_float(1u);
       return;
     }
     for (int i = 0; i < 64; ++i) {

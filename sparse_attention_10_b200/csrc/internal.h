@@ -53,6 +53,7 @@ struct SelectLaunch {
   int cap;
   const unsigned long long* cand;
   const int* cand_n;
+  const float* tau;      // per-row threshold (zero-mode rows are marked by its bits)
   int32_t* indices;
   int* fb_rows;          // [L] rows that need the exact fallback
   int* counters;         // [0] fallback rows, [1] overflow rows, [2] candidates

@@ -28,6 +28,7 @@ namespace dsa {
 namespace {
 
 constexpr int kSelThreads = 256;
+constexpr uint32_t kZeroModeTauBits = 1u;  // tau of a row whose threshold is "score > 0"
 
 __device__ __forceinline__ void block_find_from_top(const unsigned int* hist, int R, int* out) {
   // Warp 0 scans the 256 bins from the top; out[0] = bin, out[1] = rank in bin.
@@ -131,28 +132,142 @@ __device__ void finish_row(KeyPtr keys, int n, int m, int top_k, int32_t* out,
   __syncthreads();
 }
 
+// ---- sort-based select of one row ----------------------------------------------------
+//
+// The filter writes each row's candidates as two lists (one per column half
+// of the indexer tile), each already in ascending key order.  The select
+// merges them into one ascending-index run, then sorts it by score with
+// stable LSD counting passes (descending digit), so equal scores keep
+// ascending index: the result is the (score desc, index asc) order, and the
+// first m entries are the answer.  Only the score bytes that differ within
+// the row get a pass.  Ranks inside a warp come from __match_any_sync, so the
+// passes use no atomics.
+
+constexpr int kSortThreads = 512;
+constexpr int kSortWarps = kSortThreads / 32;
+constexpr int kSortMaxSlots = 11;                                  // items per lane per pass
+constexpr int kSortCap = kSortWarps * 32 * kSortMaxSlots;          // 5632 keys per row
+
+__device__ __forceinline__ uint32_t key_index(unsigned long long k) {
+  return 0xFFFFFFFFu - static_cast<uint32_t>(k);
+}
+
+// Merge two ascending-index runs a[0, na) and b[0, nb) into out (merge path).
+__device__ void merge_by_index(const unsigned long long* a, int na, const unsigned long long* b,
+                               int nb, unsigned long long* out) {
+  const int n = na + nb;
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int p0 = min(n, static_cast<int>(threadIdx.x) * per), p1 = min(n, p0 + per);
+  if (p0 >= p1) return;
+  int lo = max(0, p0 - nb), hi = min(p0, na);
+  while (lo < hi) {  // smallest i such that a[i] does not precede b[p0 - i - 1]
+    const int i = (lo + hi) >> 1;
+    if (key_index(a[i]) < key_index(b[p0 - i - 1]))
+      lo = i + 1;
+    else
+      hi = i;
+  }
+  int i = lo, j = p0 - lo;
+  for (int p = p0; p < p1; ++p) {
+    const bool take_a = j >= nb || (i < na && key_index(a[i]) < key_index(b[j]));
+    out[p] = take_a ? a[i++] : b[j++];
+  }
+}
+
+// Stable pass: out = in ordered by byte (key >> shift) & 255, descending.
+__device__ void radix_pass_desc(const unsigned long long* in, unsigned long long* out, int n,
+                                int shift, uint32_t* cnt /*[warps][256]*/, uint32_t* base /*[256]*/) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = (n + kSortWarps * 32 - 1) / (kSortWarps * 32) * 32;  // items per warp
+  const int slots = chunk / 32;
+  uint32_t* wc = cnt + warp * 256;
+  for (int d = lane; d < 256; d += 32) wc[d] = 0;
+  __syncwarp();
+  const uint32_t lt = (1u << lane) - 1u;
+  unsigned long long v[kSortMaxSlots];
+  uint32_t dg[kSortMaxSlots], rk[kSortMaxSlots];
+#pragma unroll
+  for (int j = 0; j < kSortMaxSlots; ++j) {
+    if (j < slots) {
+      const int i = warp * chunk + j * 32 + lane;
+      const bool ok = i < n;
+      v[j] = ok ? in[i] : 0ull;
+      const uint32_t d = ok ? 255u - static_cast<uint32_t>((v[j] >> shift) & 255u) : 256u;
+      dg[j] = d;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
+      const uint32_t before = ok ? wc[d] : 0u;
+      rk[j] = before + __popc(peers & lt);
+      __syncwarp();
+      if (ok && lane == __ffs(peers) - 1) wc[d] = before + __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 256) {  // per digit: warp-exclusive prefix, digit total
+    const int d = threadIdx.x;
+    uint32_t run = 0;
+    for (int w = 0; w < kSortWarps; ++w) {
+      const uint32_t c = cnt[w * 256 + d];
+      cnt[w * 256 + d] = run;
+      run += c;
+    }
+    base[d] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive scan of the 256 digit totals
+    uint32_t loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      loc[q] = base[lane * 8 + q];
+      sum += loc[q];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t ex = incl - sum;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      base[lane * 8 + q] = ex;
+      ex += loc[q];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kSortMaxSlots; ++j) {
+    if (j < slots && dg[j] < 256u) out[base[dg[j]] + cnt[warp * 256 + dg[j]] + rk[j]] = v[j];
+  }
+  __syncthreads();
+}
+
 struct SelParams {
   int64_t L;
   int top_k, cap;
   const unsigned long long* cand;
   const int* cand_n;
+  const float* tau;
   int32_t* indices;
   int* fb_rows;
   int* counters;
 };
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) {
+__global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long sel_smem[];
-  unsigned long long* keys = sel_smem;                        // [2 * cap]
-  unsigned long long* sel = keys + 2 * p.cap;                 // [top_k rounded to pow2]
-  unsigned int* hist = reinterpret_cast<unsigned int*>(sel + next_pow2(max(p.top_k, 2)));
-  int* shared2 = reinterpret_cast<int*>(hist + 256);
+  unsigned long long* bufA = sel_smem;                          // [kSortCap]
+  unsigned long long* bufB = bufA + kSortCap;                   // [kSortCap]
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(bufB + kSortCap); // [warps][256] (also the bitmap)
+  uint32_t* base = cnt + kSortWarps * 256;                      // [256]
+  uint32_t* misc = base + 256;                                  // [8]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
     const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
-    const bool overflow = n0 > p.cap || n1 > p.cap;
+    const bool overflow = n0 > p.cap || n1 > p.cap || n0 + n1 > kSortCap;
+    const bool zero_mode = __float_as_uint(p.tau[t]) == kZeroModeTauBits;
     const int n = n0 + n1;
-    if (overflow || n < m) {
+    if (overflow || (!zero_mode && n < m)) {
       if (threadIdx.x == 0) {
         const int pos = atomicAdd(&p.counters[0], 1);
         p.fb_rows[pos] = static_cast<int>(t);
@@ -160,13 +275,101 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SelParams p) 
       }
       continue;
     }
-    if (threadIdx.x == 0) atomicAdd(&p.counters[2], n);
+    if (threadIdx.x == 0) {
+      atomicAdd(&p.counters[2], n);
+      misc[0] = 0u;           // OR of score words
+      misc[1] = 0xFFFFFFFFu;  // AND of score words
+      misc[2] = 0u;           // positive scores
+    }
     const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
     const unsigned long long* c1 = c0 + p.cap;
-    for (int i = threadIdx.x; i < n0; i += blockDim.x) keys[i] = c0[i];
-    for (int i = threadIdx.x; i < n1; i += blockDim.x) keys[n0 + i] = c1[i];
+    for (int i = threadIdx.x; i < n0; i += blockDim.x) bufA[i] = c0[i];
+    for (int i = threadIdx.x; i < n1; i += blockDim.x) bufA[n0 + i] = c1[i];
     __syncthreads();
-    finish_row(keys, n, m, p.top_k, p.indices + t * p.top_k, sel, hist, shared2);
+    merge_by_index(bufA, n0, bufA + n0, n1, bufB);
+    __syncthreads();
+    uint32_t o = 0u, a = 0xFFFFFFFFu, pos = 0u;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t hi = static_cast<uint32_t>(bufB[i] >> 32);
+      o |= hi;
+      a &= hi;
+      pos += hi != 0u;
+    }
+    o = __reduce_or_sync(0xFFFFFFFFu, o);
+    a = __reduce_and_sync(0xFFFFFFFFu, a);
+    pos = __reduce_add_sync(0xFFFFFFFFu, pos);
+    if (lane == 0) {
+      atomicOr(&misc[0], o);
+      atomicAnd(&misc[1], a);
+      atomicAdd(&misc[2], pos);
+    }
+    __syncthreads();
+    const uint32_t vary = misc[0] ^ misc[1];
+    const int npos = static_cast<int>(misc[2]);
+    unsigned long long* cur = bufB;
+    unsigned long long* nxt = bufA;
+    for (int byte = 0; byte < 4; ++byte) {
+      if ((vary >> (8 * byte)) & 255u) {
+        radix_pass_desc(cur, nxt, n, 32 + 8 * byte, cnt, base);
+        unsigned long long* tmp = cur;
+        cur = nxt;
+        nxt = tmp;
+      }
+    }
+    int32_t* out = p.indices + t * p.top_k;
+    if (!zero_mode || npos >= m) {
+      for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
+        out[i] = i < m ? static_cast<int32_t>(key_index(cur[i])) : -1;
+    } else {
+      // Every positive score is a candidate; the rest of the row ranks the
+      // zero scores by ascending key index.  Within keys [0, R) there are at
+      // least m - npos zeros.
+      const int R = static_cast<int>(min64(t + 1, static_cast<int64_t>(m) + npos));
+      const int words = (R + 31) / 32;
+      uint32_t* bm = cnt;
+      for (int wd = threadIdx.x; wd < words; wd += blockDim.x) bm[wd] = 0u;
+      __syncthreads();
+      for (int i = threadIdx.x; i < npos; i += blockDim.x) {
+        const uint32_t s = key_index(cur[i]);
+        if (s < static_cast<uint32_t>(R)) atomicOr(&bm[s >> 5], 1u << (s & 31));
+        out[i] = static_cast<int32_t>(s);
+      }
+      __syncthreads();
+      // zero count per word, exclusive scan over words (words <= 128)
+      uint32_t z = 0u;
+      if (threadIdx.x < words) {
+        const int wd = threadIdx.x;
+        const uint32_t valid = (wd * 32 + 32 <= R) ? 0xFFFFFFFFu : ((1u << (R - wd * 32)) - 1u);
+        z = __popc(~bm[wd] & valid);
+      }
+      if (threadIdx.x < 128) {
+        uint32_t incl = z;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        if (lane == 31) base[warp] = incl;
+        __syncwarp();
+        base[8 + threadIdx.x] = incl - z;  // exclusive within the warp
+      }
+      __syncthreads();
+      if (threadIdx.x < words) {
+        const int wd = threadIdx.x;
+        uint32_t rank = base[8 + wd];
+        for (int w2 = 0; w2 < warp; ++w2) rank += base[w2];
+        const uint32_t valid = (wd * 32 + 32 <= R) ? 0xFFFFFFFFu : ((1u << (R - wd * 32)) - 1u);
+        uint32_t zeros = ~bm[wd] & valid;
+        while (zeros) {
+          const int b = __ffs(zeros) - 1;
+          zeros &= zeros - 1u;
+          if (rank < static_cast<uint32_t>(m - npos)) out[npos + rank] = wd * 32 + b;
+          ++rank;
+        }
+      }
+      for (int i = m + threadIdx.x; i < p.top_k; i += blockDim.x) out[i] = -1;
+    }
+    __syncthreads();
   }
 }
 
@@ -262,13 +465,14 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
 
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
-  SelParams p{a.L, a.top_k, a.cap, a.cand, a.cand_n, a.indices, a.fb_rows, a.counters};
-  const size_t smem = (2 * static_cast<size_t>(a.cap) + P) * 8 + 256 * 4 + 16;
+  if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
+  SelParams p{a.L, a.top_k, a.cap, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
+  const size_t smem = 2 * static_cast<size_t>(kSortCap) * 8 + (kSortWarps * 256 + 256 + 8) * 4;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return DSA_ERR_CUDA;
-  const int grid = static_cast<int>(std::min<int64_t>(a.L, 4 * num_sms()));
-  select_kernel<<<grid, kSelThreads, smem, stream>>>(p);
+  const int grid = static_cast<int>(std::min<int64_t>(a.L, 2 * num_sms()));
+  select_kernel<<<grid, kSortThreads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
 
   FbParams f{a.L, a.top_k, a.q_idx, a.k_idx, a.esize, a.d, a.scale, a.fb_rows, a.counters,
