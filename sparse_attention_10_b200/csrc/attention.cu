@@ -89,13 +89,33 @@ struct AttnParams {
 };
 
 template <int D>
+struct AttnSmem {
+  static constexpr int kRowQ = 2 * D + 16;            // padded Q row (bytes)
+  static constexpr int kRowKV = 2 * D;                // K/V rows are XOR-swizzled, not padded
+  static constexpr int kTile = kKeysPerTile * kRowKV; // one K (or V) tile
+  static constexpr int kStages = D == 64 ? 4 : 3;
+  static constexpr int kQ = 16 * kRowQ;
+  static constexpr int kIds = DSA_MAX_TOP_K * 4;
+  static constexpr int kBytes = kQ + kIds + kStages * 2 * kTile;
+};
+
+// Byte offset of 16-byte chunk c of row r in a swizzled K/V tile: the chunk
+// index is XORed with the row's low three bits, so the eight rows an
+// ldmatrix reads at one logical chunk fall in eight different bank groups.
+template <int D>
+__device__ __forceinline__ uint32_t kv_off(int r, int c) {
+  return static_cast<uint32_t>(r * (2 * D) + ((c ^ (r & 7)) << 4));
+}
+
+template <int D>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) {
-  constexpr int RS = 2 * D + 16;                 // padded row stride (bytes) of every tile
+  using SM = AttnSmem<D>;
   constexpr int PIECES = D / 8;                  // 16-byte pieces per row
-  constexpr int TILE = kKeysPerTile * RS;        // bytes of one K (or V) tile
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* sQ = smem;                            // 16 rows
-  uint8_t* sKV = smem + 16 * RS;                 // [2 stages][K tile, V tile]
+  constexpr int NST = SM::kStages;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sQ = smem;                                         // 16 padded rows
+  int32_t* sIds = reinterpret_cast<int32_t*>(smem + SM::kQ);  // this item's key list
+  uint8_t* sKV = smem + SM::kQ + SM::kIds;                    // [stages][K tile, V tile]
   const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
@@ -115,43 +135,54 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     }
     const int per = (count + p.nsplit - 1) / p.nsplit;
     const int begin = min(count, sp * per), end = min(count, begin + per);
-    const int32_t* ids = p.idx + q * p.ld_idx;
+    const int n = end - begin;
+    const int32_t* ids = p.idx + q * p.ld_idx + begin;
     // rows a query may read: its causal prefix (prefill) or its sequence (decode)
     const int row_limit = p.seq_start ? static_cast<int>(p.seq_start[q + 1] - row_base)
                                       : static_cast<int>(min64(q + 1, 0x7FFFFFFF));
     const __nv_bfloat16* Kb = p.K + row_base * D;
     const __nv_bfloat16* Vb = p.V + row_base * D;
 
-    // Q rows (heads >= H are zero).
+    // Q rows (heads >= H are zero) and this item's key list, clamped.
     for (int i = tid; i < 16 * PIECES; i += kAttnThreads) {
       const int r = i / PIECES, c = i % PIECES;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (r < p.H) v = *reinterpret_cast<const uint4*>(p.Q + (q * p.H + r) * D + c * 8);
-      *reinterpret_cast<uint4*>(sQ + r * RS + c * 16) = v;
+      *reinterpret_cast<uint4*>(sQ + r * SM::kRowQ + c * 16) = v;
     }
+    for (int i = tid; i < n; i += kAttnThreads) {
+      const int s = ids[i];
+      sIds[i] = (s >= 0 && s < row_limit) ? s : -1;
+    }
+    __syncthreads();
 
-    const int ntiles = (end - begin + kKeysPerTile - 1) / kKeysPerTile;
+    const int ntiles = (n + kKeysPerTile - 1) / kKeysPerTile;
+    // Warp w copies key rows w, w+4, ...; its 32 lanes take the 16-byte pieces
+    // of one K row and one V row (coalesced 2D-byte rows).
     auto issue = [&](int tile) {
-      const uint32_t st = sKVa + (tile & 1) * 2 * TILE;
-      for (int i = tid; i < kKeysPerTile * 2 * PIECES; i += kAttnThreads) {
-        const int r = i / (2 * PIECES), rem = i % (2 * PIECES);
-        const int kv = rem / PIECES, c = rem % PIECES;
-        const int j = begin + tile * kKeysPerTile + r;
-        int s = j < end ? ids[j] : -1;
-        if (s >= row_limit) s = -1;  // never read past the sequence
-        const __nv_bfloat16* src = (kv ? Vb : Kb) + static_cast<int64_t>(s < 0 ? 0 : s) * D + c * 8;
-        cp_async16(st + kv * TILE + r * RS + c * 16, src, s < 0 ? 0u : 16u);
+      if (tile < ntiles) {
+        const uint32_t st = sKVa + (tile % NST) * 2 * SM::kTile;
+#pragma unroll
+        for (int u = 0; u < kKeysPerTile * 2 * PIECES / kAttnThreads; ++u) {
+          const int i = tid + u * kAttnThreads;
+          const int r = i / (2 * PIECES), rem = i % (2 * PIECES);
+          const int kv = rem / PIECES, c = rem % PIECES;
+          const int j = tile * kKeysPerTile + r;
+          const int s = j < n ? sIds[j] : -1;
+          const __nv_bfloat16* src = (kv ? Vb : Kb) + static_cast<int64_t>(s < 0 ? 0 : s) * D + c * 8;
+          cp_async16(st + kv * SM::kTile + kv_off<D>(r, c), src, s < 0 ? 0u : 16u);
+        }
       }
-      cp_async_commit();
+      cp_async_commit();  // possibly empty: keeps one group per tile
     };
-    if (ntiles > 0) issue(0);
-    __syncthreads();  // Q visible
+#pragma unroll
+    for (int t = 0; t < NST - 1; ++t) issue(t);
 
     uint32_t qa[D / 16][4];
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const int r = (lane & 7) + ((lane >> 3) & 1) * 8, c = kk * 16 + (lane >> 4) * 8;
-      ldsm_x4(sQa + r * RS + c * 2, qa[kk]);
+      ldsm_x4(sQa + r * SM::kRowQ + c * 2, qa[kk]);
     }
     float o[D / 8][4];
 #pragma unroll
@@ -159,32 +190,28 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
 
     for (int tile = 0; tile < ntiles; ++tile) {
-      if (tile + 1 < ntiles) {
-        issue(tile + 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncthreads();
-      const uint32_t sK = sKVa + (tile & 1) * 2 * TILE + warp * 16 * RS;
-      const uint32_t sV = sK + TILE;
+      cp_async_wait<NST - 2>();   // this tile's copies (issued NST-1 tiles ago) are done
+      __syncthreads();            // ... for every thread; the oldest stage is free again
+      issue(tile + NST - 1);
+      const uint32_t sK = sKVa + (tile % NST) * 2 * SM::kTile;
+      const uint32_t sV = sK + SM::kTile;
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t b[4];
-        const int r = (lane & 7) + (lane >> 4) * 8, c = kk * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x4(sK + r * RS + c * 2, b);
+        const int r = warp * 16 + (lane & 7) + (lane >> 4) * 8, c = kk * 2 + ((lane >> 3) & 1);
+        ldsm_x4(sK + kv_off<D>(r, c), b);
         mma16816(s[0], qa[kk], b[0], b[1]);
         mma16816(s[1], qa[kk], b[2], b[3]);
       }
-      // scale (log2 domain) and mask keys past the end of this split
-      const int key0 = begin + tile * kKeysPerTile + warp * 16;
+      // scale (log2 domain) and mask keys past the end of this item's list
+      const int key0 = tile * kKeysPerTile + warp * 16;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = key0 + nt * 8 + tig * 2 + (e & 1);
-          s[nt][e] = j < end ? s[nt][e] * p.scale_log2 : -INFINITY;
+          s[nt][e] = j < n ? s[nt][e] * p.scale_log2 : -INFINITY;
         }
       float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
       float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
@@ -194,6 +221,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
       const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
       const float r0 = n0 == -INFINITY ? 0.0f : n0, r1 = n1 == -INFINITY ? 0.0f : n1;
+      const bool same = n0 == m0 && n1 == m1;
       const float c0 = fast_exp2(m0 - r0), c1 = fast_exp2(m1 - r1);
       m0 = n0;
       m1 = n1;
@@ -205,14 +233,21 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
         pr[nt][2] = fast_exp2(s[nt][2] - r1);
         pr[nt][3] = fast_exp2(s[nt][3] - r1);
       }
-      l0 = l0 * c0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
-      l1 = l1 * c1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+      const float ps0 = pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
+      const float ps1 = pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];
+      if (__all_sync(0xFFFFFFFFu, same)) {   // no row max moved: nothing to rescale
+        l0 += ps0;
+        l1 += ps1;
+      } else {
+        l0 = l0 * c0 + ps0;
+        l1 = l1 * c1 + ps1;
 #pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        o[i][0] *= c0;
-        o[i][1] *= c0;
-        o[i][2] *= c1;
-        o[i][3] *= c1;
+        for (int i = 0; i < D / 8; ++i) {
+          o[i][0] *= c0;
+          o[i][1] *= c0;
+          o[i][2] *= c1;
+          o[i][3] *= c1;
+        }
       }
       uint32_t pa[4];
       pa[0] = pack_bf16(pr[0][0], pr[0][1]);
@@ -222,13 +257,14 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
 #pragma unroll
       for (int dt = 0; dt < D / 16; ++dt) {
         uint32_t b[4];
-        const int r = (lane & 7) + ((lane >> 3) & 1) * 8, c = dt * 16 + (lane >> 4) * 8;
-        ldsm_x4_t(sV + r * RS + c * 2, b);
+        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = dt * 2 + (lane >> 4);
+        ldsm_x4_t(sV + kv_off<D>(r, c), b);
         mma16816(o[2 * dt], pa, b[0], b[1]);
         mma16816(o[2 * dt + 1], pa, b[2], b[3]);
       }
-      __syncthreads();  // this stage is refilled two tiles later
     }
+    cp_async_wait<0>();
+    __syncthreads();  // all warps done with the tiles: the stage area becomes the merge area
 
     // ---- merge the four warps' partial states
     l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
@@ -309,9 +345,8 @@ template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p{a.Q, a.K, a.V, a.idx, a.ld_idx, a.nq, a.H, a.scale_log2, a.top_k, a.seq_start,
                a.nsplit, a.O, a.part, a.invalid};
-  constexpr int RS = 2 * D + 16;
-  const size_t smem = static_cast<size_t>(16 + 2 * 2 * kKeysPerTile) * RS;
-  static_assert((16 + 2 * 2 * kKeysPerTile) * (2 * D + 16) >= (4 * 16 * 2 + 4 * 16 * D) * 4,
+  const size_t smem = AttnSmem<D>::kBytes;
+  static_assert(AttnSmem<D>::kStages * 2 * AttnSmem<D>::kTile >= (4 * 16 * 2 + 4 * 16 * D) * 4,
                 "merge area must fit in the tiles");
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));

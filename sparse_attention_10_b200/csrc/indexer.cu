@@ -45,6 +45,7 @@ constexpr uint32_t kTileA = kBM * 32;   // bytes of one 32-byte K slice of the A
 constexpr uint32_t kTileB = kBN * 32;   // bytes of one 32-byte K slice of a B tile
 
 struct Params {
+  const void* k_idx;
   int64_t Lq, Lk;
   int nkb, stages;
   uint32_t off_b, off_stage, off_bar;
@@ -108,6 +109,38 @@ __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
   return (f > 0.0f ? acc_bits : 0u) >> 16;  // non-negative float bits are monotone
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+// Sample tile j of query tile qt: 256 key rows spread evenly over the keys
+// below the band [r0 - 128, r0 + 128) (stratified, so every region of the
+// prefix is represented), copied into the same 32-byte-swizzled K-major
+// layout the TMA path writes: row r, 16-byte chunk c of 32-byte slice b goes
+// to b * 8 KB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4).  All 32 lanes copy;
+// the copies are complete and visible to the tensor core on return.
+__device__ __forceinline__ void gather_sample_tile(const Params& p, const uint8_t* k_idx,
+                                                   int64_t qt, int j, int nt, uint32_t dst,
+                                                   int lane) {
+  const int pieces = 2 * p.nkb;                 // 16-byte pieces per row
+  const int rows_per_iter = 32 / pieces;        // nkb <= 16
+  const int rsub = lane / pieces, q = lane % pieces;
+  const int b = q >> 1, c = q & 1;
+  const int64_t span = qt * kBM - 128;          // keys [0, span) are below the band
+  const int64_t ns = static_cast<int64_t>(nt) * kBN;
+  const int64_t row_bytes = static_cast<int64_t>(p.nkb) * 32;
+  if (rsub < rows_per_iter) {
+    for (int r = rsub; r < kBN; r += rows_per_iter) {
+      const int64_t key = (static_cast<int64_t>(j) * kBN + r) * span / ns;
+      cp_async16(dst + b * kTileB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4),
+                 k_idx + key * row_bytes + q * 16);
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+}
+
 template <int ESIZE>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -159,8 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // ------------------------------------------------------------ producer
+    // Lane 0 issues the TMA copies and barrier operations.  In sample mode the
+    // whole warp gathers the sampled key rows with cp.async instead.
+    const bool gather = p.mode == kModeSample;
+    if (gather || lane == 0) {
       uint32_t it = 0, item_it = 0;
       bool ok = true;
       for (int round = 0; ok; ++round) {
@@ -169,40 +205,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t qt = item_qtile(p, item);
         const int nt = item_ntiles(p, qt);
         if (nt == 0) continue;
-        if (!mbar_wait(bar(A_EMPTY), (item_it & 1) ^ 1, p.limit_ns, abort_flag)) {
-          ok = false;
-          break;
+        if (lane == 0) {
+          ok = mbar_wait(bar(A_EMPTY), (item_it & 1) ^ 1, p.limit_ns, abort_flag);
+          if (ok) {
+            mbar_arrive_expect_tx(bar(A_FULL), p.nkb * kTileA);
+            for (int b = 0; b < p.nkb; ++b)
+              tma_load_2d(sA + b * kTileA, &tmQ, b * (32 / ESIZE), static_cast<int>(qt * kBM),
+                          bar(A_FULL));
+          }
         }
-        mbar_arrive_expect_tx(bar(A_FULL), p.nkb * kTileA);
-        for (int b = 0; b < p.nkb; ++b)
-          tma_load_2d(sA + b * kTileA, &tmQ, b * (32 / ESIZE), static_cast<int>(qt * kBM),
-                      bar(A_FULL));
+        if (gather) ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
         ++item_it;
         for (int j = 0; j < nt; ++j) {
           const uint32_t s = it % S, ph = (it / S) & 1;
-          if (!mbar_wait(bar(EMPTY + s), ph ^ 1, p.limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
-          const int kt = item_ktile(p, qt, j, nt);
+          if (lane == 0) ok = mbar_wait(bar(EMPTY + s), ph ^ 1, p.limit_ns, abort_flag);
+          if (gather) ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
           const uint32_t dst = sB + s * stage_bytes;
-          for (int b = 0; b < p.nkb; ++b)
-            tma_load_2d(dst + b * kTileB, &tmK, b * (32 / ESIZE), kt * kBN, bar(FULL + s));
+          if (!gather) {
+            mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
+            const int kt = item_ktile(p, qt, j, nt);
+            for (int b = 0; b < p.nkb; ++b)
+              tma_load_2d(dst + b * kTileB, &tmK, b * (32 / ESIZE), kt * kBN, bar(FULL + s));
+          } else {
+            gather_sample_tile(p, static_cast<const uint8_t*>(p.k_idx), qt, j, nt, dst, lane);
+            if (lane == 0) mbar_arrive(bar(FULL + s));
+          }
           ++it;
         }
       }
-      const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
-      if (ok) {
-        // Every stage still held is released by an MMA commit; wait for those
-        // arrivals so none lands after the CTA exits.
-        for (uint32_t i = first; i < it; ++i)
-          mbar_wait(bar(EMPTY + i % S), (i / S) & 1, p.limit_ns, nullptr);
-      } else {
-        // Aborted: wait for the data of every copy still in flight.
-        for (uint32_t i = first; i < it; ++i)
-          mbar_wait(bar(FULL + i % S), (i / S) & 1, p.limit_ns, nullptr);
-        if (item_it) mbar_wait(bar(A_FULL), (item_it - 1) & 1, p.limit_ns, nullptr);
+      if (lane == 0) {
+        const uint32_t first = it > static_cast<uint32_t>(S) ? it - S : 0;
+        if (ok) {
+          // Every stage still held is released by an MMA commit; wait for those
+          // arrivals so none lands after the CTA exits.
+          for (uint32_t i = first; i < it; ++i)
+            mbar_wait(bar(EMPTY + i % S), (i / S) & 1, p.limit_ns, nullptr);
+        } else {
+          // Aborted: wait for the data of every copy still in flight.
+          for (uint32_t i = first; i < it; ++i)
+            mbar_wait(bar(FULL + i % S), (i / S) & 1, p.limit_ns, nullptr);
+          if (item_it) mbar_wait(bar(A_FULL), (item_it - 1) & 1, p.limit_ns, nullptr);
+        }
       }
     }
   } else if (warp == 1) {
@@ -502,6 +547,7 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   if (stages < 1) return DSA_ERR_UNSUPPORTED;
 
   Params p{};
+  p.k_idx = a.k_idx;
   p.Lq = a.Lq;
   p.Lk = a.Lk;
   p.nkb = nkb;
