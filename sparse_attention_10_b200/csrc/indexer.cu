@@ -117,8 +117,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 // below the band [r0 - 128, r0 + 128) (stratified, so every region of the
 // prefix is represented), copied into the same 32-byte-swizzled K-major
 // layout the TMA path writes: row r, 16-byte chunk c of 32-byte slice b goes
-// to b * 8 KB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4).  All 32 lanes copy;
-// the copies are complete and visible to the tensor core on return.
+// to b * 8 KB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4).  All 32 lanes issue
+// cp.async copies and commit them as one group; sample_tile_done() completes
+// an older group.
 __device__ __forceinline__ void gather_sample_tile(const Params& p, const uint8_t* k_idx,
                                                    int64_t qt, int j, int nt, uint32_t dst,
                                                    int lane) {
@@ -136,7 +137,14 @@ __device__ __forceinline__ void gather_sample_tile(const Params& p, const uint8_
                  k_idx + key * row_bytes + q * 16);
     }
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Waits until at most `pending` gather groups of this lane are in flight, then
+// makes the landed rows visible to the tensor core (async proxy) for the warp.
+template <int PENDING>
+__device__ __forceinline__ void sample_tile_done() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
 }
@@ -229,10 +237,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < p.nkb; ++b)
               tma_load_2d(dst + b * kTileB, &tmK, b * (32 / ESIZE), kt * kBN, bar(FULL + s));
           } else {
+            // Two tiles in flight: issue tile j, then publish tile j-1.  With a
+            // single stage, tile j's slot frees only after tile j-1 is consumed,
+            // so publish each tile right away.
             gather_sample_tile(p, static_cast<const uint8_t*>(p.k_idx), qt, j, nt, dst, lane);
-            if (lane == 0) mbar_arrive(bar(FULL + s));
+            if (S == 1) {
+              sample_tile_done<0>();
+              if (lane == 0) mbar_arrive(bar(FULL + s));
+            } else if (j > 0) {
+              sample_tile_done<1>();
+              if (lane == 0) mbar_arrive(bar(FULL + (it - 1) % S));
+            }
           }
           ++it;
+        }
+        if (gather) {  // publish the item's last tile (or drain after an abort)
+          sample_tile_done<0>();
+          if (ok && S > 1 && lane == 0) mbar_arrive(bar(FULL + (it - 1) % S));
         }
       }
       if (lane == 0) {

@@ -128,6 +128,19 @@ def test_prefill_bf16_index(dsa):
     compare(x, "bf16", 300, idx, O)
 
 
+def test_prefill_bf16_index_dim_256_single_stage(dsa):
+    # 512-byte index rows leave room for one pipeline stage in the indexer.
+    x = small_inputs(1500, 256, 2, 64, idx_dtype="bf16", seed=13)
+    idx, O, _ = run_prefill(dsa, x, 128)
+    compare(x, "bf16", 128, idx, O)
+
+
+def test_prefill_fp8_index_dim_256(dsa):
+    x = small_inputs(1700, 256, 2, 64, seed=14)
+    idx, O, _ = run_prefill(dsa, x, 96)
+    compare(x, "fp8", 96, idx, O)
+
+
 def test_prefill_many_ties(dsa):
     # Index values in {-1, 0, 1}: scores take few values, so ties cross the k-th place.
     x = small_inputs(3000, 32, 2, 64, seed=8, lo=-1, hi=1)
