@@ -129,11 +129,19 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
   __syncthreads();
-  for (int64_t s = c0 + threadIdx.x; s < c1; s += blockDim.x) {
-    float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, base + s, p.d), p.scale);
-    sc = sc > 0.0f ? sc : 0.0f;
-    p.scores[base + s] = sc;
-    atomicAdd(&hist[__float_as_uint(sc) >> 20], 1u);
+  // Zero scores are not counted (the select recovers them as len - sum of
+  // bins); lanes that hit the same bin add once through their leader.
+  for (int64_t s0 = c0; s0 < c1; s0 += blockDim.x) {
+    const int64_t s = s0 + threadIdx.x;
+    uint32_t bin = 0;
+    if (s < c1) {
+      float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, base + s, p.d), p.scale);
+      sc = sc > 0.0f ? sc : 0.0f;
+      p.scores[base + s] = sc;
+      bin = __float_as_uint(sc) >> 20;
+    }
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+    if (bin != 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
@@ -235,11 +243,17 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   const float* sc = p.scores + base;
   const unsigned int* hist = p.hist + static_cast<int64_t>(b) * kHistBins;
 
-  // Bin of the m-th best score (bins scanned from the top by warp 0).
+  // Bin of the m-th best score (bins scanned from the top by warp 0).  Bin 0
+  // (score +0) is not counted by the scan: every key not in a higher bin.
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     unsigned int local = 0;
-    for (int i = 0; i < kHistBins / 32; ++i) local += hist[kHistBins - 1 - (kHistBins / 32) * lane - i];
+    for (int i = 0; i < kHistBins / 32; ++i) {
+      const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
+      if (bb > 0) local += hist[bb];
+    }
+    const unsigned int above0 = __reduce_add_sync(0xFFFFFFFFu, local);
+    if (lane == 31) local += static_cast<unsigned int>(n) - above0;
     unsigned int incl = local;
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
@@ -251,7 +265,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
       unsigned int run = incl - local;
       for (int i = 0; i < kHistBins / 32; ++i) {
         const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
-        run += hist[bb];
+        run += bb > 0 ? hist[bb] : static_cast<unsigned int>(n) - above0;
         if (run >= static_cast<unsigned int>(m)) {
           sh[0] = bb;
           sh[1] = static_cast<int>(run);  // keys in bins >= bb

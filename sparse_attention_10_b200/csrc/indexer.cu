@@ -127,12 +127,14 @@ __device__ __forceinline__ void gather_sample_tile(const Params& p, const uint8_
   const int rows_per_iter = 32 / pieces;        // nkb <= 16
   const int rsub = lane / pieces, q = lane % pieces;
   const int b = q >> 1, c = q & 1;
-  const int64_t span = qt * kBM - 128;          // keys [0, span) are below the band
-  const int64_t ns = static_cast<int64_t>(nt) * kBN;
+  const uint64_t span = static_cast<uint64_t>(qt * kBM - 128);  // keys [0, span) below the band
+  const uint64_t ns = static_cast<uint64_t>(nt) * kBN;           // ns <= span
+  const uint64_t step16 = (span << 16) / ns;                     // span / ns in 48.16 fixed point
   const int64_t row_bytes = static_cast<int64_t>(p.nkb) * 32;
   if (rsub < rows_per_iter) {
     for (int r = rsub; r < kBN; r += rows_per_iter) {
-      const int64_t key = (static_cast<int64_t>(j) * kBN + r) * span / ns;
+      // key = floor(i * span / ns) up to the fixed-point truncation: < span, nondecreasing
+      const int64_t key = static_cast<int64_t>((static_cast<uint64_t>(j * kBN + r) * step16) >> 16);
       cp_async16(dst + b * kTileB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4),
                  k_idx + key * row_bytes + q * 16);
     }
