@@ -34,6 +34,9 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Bound on a single device-side wait (nanoseconds).
+__device__ __forceinline__ uint64_t wait_limit_ns_device() { return 2000000000ull; }
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -323,6 +323,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   at.Q = static_cast<const __nv_bfloat16*>(Q);
   at.K = static_cast<const __nv_bfloat16*>(K);
   at.V = static_cast<const __nv_bfloat16*>(V);
+  at.kv_rows = L;
   at.idx = indices;
   at.ld_idx = top_k;
   at.nq = L;
@@ -397,6 +398,7 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
   at.Q = static_cast<const __nv_bfloat16*>(Q);
   at.K = static_cast<const __nv_bfloat16*>(K);
   at.V = static_cast<const __nv_bfloat16*>(V);
+  at.kv_rows = total_rows;
   at.idx = idx;
   at.ld_idx = top_k;
   at.nq = B;

@@ -74,6 +74,7 @@ struct AttnLaunch {
   const __nv_bfloat16* Q;      // [nq, H, D]
   const __nv_bfloat16* K;      // [rows, D]
   const __nv_bfloat16* V;
+  int64_t kv_rows;             // rows of K and V
   const int32_t* idx;          // [nq, ld_idx]
   int ld_idx;
   int64_t nq;
