@@ -14,8 +14,6 @@
 // mma.sync.  The four warps' partial (max, sum, O) are merged at the end.
 // With more than one split per query (decode), each split writes its
 // partial state and a combine kernel merges them (log-sum-exp).
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 
 #include "common.cuh"
@@ -93,70 +91,38 @@ struct AttnParams {
 template <int D>
 struct AttnSmem {
   static constexpr int kRowQ = 2 * D + 16;            // padded Q row (bytes)
-  static constexpr int kHalves = D / 64;              // 128-byte column blocks of a K/V row
-  static constexpr int kHalfTile = kKeysPerTile * 128;
-  static constexpr int kTile = kHalves * kHalfTile;   // one K (or V) tile
+  static constexpr int kRowKV = 2 * D;                // K/V rows are XOR-swizzled, not padded
+  static constexpr int kTile = kKeysPerTile * kRowKV; // one K (or V) tile
   static constexpr int kStages = D == 64 ? 4 : 3;
   static constexpr int kQ = 16 * kRowQ;
   static constexpr int kIds = DSA_MAX_TOP_K * 4;
-  static constexpr int kBars = 64;
   static constexpr int kMergeRow = D + 8;             // padded merge rows (floats)
-  static constexpr int kBytes = 1024 + kStages * 2 * kTile + kQ + kIds + kBars;
+  static constexpr int kBytes = kQ + kIds + kStages * 2 * kTile;
 };
 
-// Byte offset of 16-byte chunk c (0 .. D/8-1) of key row r in a K/V tile.
-// A tile is stored as 128-byte column blocks (dims 64h .. 64h+63), each a
-// 64-row array with the 128-byte swizzle the tensor copy applies: chunk
-// (c mod 8) of row r sits at position (c mod 8) ^ (r mod 8), so the eight
-// rows an ldmatrix reads at one logical chunk fall in eight bank groups.
+// Byte offset of 16-byte chunk c of row r in a swizzled K/V tile: the chunk
+// index is XORed with the row's low three bits, so the eight rows an
+// ldmatrix reads at one logical chunk fall in eight different bank groups.
+template <int D>
 __device__ __forceinline__ uint32_t kv_off(int r, int c) {
-  return static_cast<uint32_t>((c >> 3) * (kKeysPerTile * 128) + r * 128 +
-                               (((c & 7) ^ (r & 7)) << 4));
-}
-
-// Four rows (y0..y3) of a 2D tensor, columns x .. x+63, into shared memory
-// (512 bytes), completion counted in bytes on `bar`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0,
-                                            int y1, int y2, int y3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
+  return static_cast<uint32_t>(r * (2 * D) + ((c ^ (r & 7)) << 4));
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                            const __grid_constant__ CUtensorMap tmV,
-                                                            const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) {
   using SM = AttnSmem<D>;
   constexpr int PIECES = D / 8;                  // 16-byte pieces per row
   constexpr int NST = SM::kStages;
-  constexpr int HALVES = SM::kHalves;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sKV = smem;                                                   // [stages][K, V]
-  uint8_t* sQ = smem + NST * 2 * SM::kTile;                              // 16 padded rows
-  int32_t* sIds = reinterpret_cast<int32_t*>(sQ + SM::kQ);               // this item's keys
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + SM::kQ + SM::kIds);  // [stages]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + NST);
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* sQ = smem;                                         // 16 padded rows
+  int32_t* sIds = reinterpret_cast<int32_t*>(smem + SM::kQ);  // this item's key list
+  uint8_t* sKV = smem + SM::kQ + SM::kIds;                    // [stages][K tile, V tile]
   const uint32_t sQa = smem_u32(sQ), sKVa = smem_u32(sKV);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;
   const int64_t n_items = p.nq * p.nsplit;
 
   if (p.invalid && *p.invalid) return;
-  if (tid == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(smem_u32(bars + i), 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    tma_prefetch_desc(&tmK);
-    tma_prefetch_desc(&tmV);
-  }
-  __syncthreads();
-  uint32_t gt = 0;  // tiles consumed by this CTA so far (stage / phase of the ring)
-
   for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int64_t q = item / p.nsplit;
     const int sp = static_cast<int>(item % p.nsplit);
@@ -175,41 +141,40 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
     // rows a query may read: its causal prefix (prefill) or its sequence (decode)
     const int row_limit = p.seq_start ? static_cast<int>(p.seq_start[q + 1] - row_base)
                                       : static_cast<int>(min64(q + 1, 0x7FFFFFFF));
+    const __nv_bfloat16* Kb = p.K + row_base * D;
+    const __nv_bfloat16* Vb = p.V + row_base * D;
 
-    // Q rows (heads >= H are zero) and this item's key rows (absolute), clamped:
-    // a padded or out-of-range entry reads the sequence's first row and is
-    // masked out of the softmax below.
+    // Q rows (heads >= H are zero) and this item's key list, clamped.
     for (int i = tid; i < 16 * PIECES; i += kAttnThreads) {
       const int r = i / PIECES, c = i % PIECES;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (r < p.H) v = *reinterpret_cast<const uint4*>(p.Q + (q * p.H + r) * D + c * 8);
       *reinterpret_cast<uint4*>(sQ + r * SM::kRowQ + c * 16) = v;
     }
-    const int ntiles = (n + kKeysPerTile - 1) / kKeysPerTile;
-    for (int i = tid; i < ntiles * kKeysPerTile; i += kAttnThreads) {
-      const int s = i < n ? ids[i] : -1;
-      sIds[i] = static_cast<int>(row_base) + ((s >= 0 && s < row_limit) ? s : 0);
+    for (int i = tid; i < n; i += kAttnThreads) {
+      const int s = ids[i];
+      sIds[i] = (s >= 0 && s < row_limit) ? s : -1;
     }
     __syncthreads();
 
-    // Warp 0 fills a stage: 64 keys x (K, V) x column blocks, 4 rows per copy.
+    const int ntiles = (n + kKeysPerTile - 1) / kKeysPerTile;
+    // Warp w copies key rows w, w+4, ...; its 32 lanes take the 16-byte pieces
+    // of one K row and one V row (coalesced 2D-byte rows).
     auto issue = [&](int tile) {
-      if (tile >= ntiles || warp != 0) return;
-      const uint32_t st = (gt + tile) % NST;
-      const uint32_t bar = smem_u32(bars + st);
-      // Order this CTA's earlier generic accesses of the stage (the previous
-      // item's merge area) before the tensor copies overwrite it.
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (lane == 0) mbar_arrive_expect_tx(bar, 2 * SM::kTile);
-      __syncwarp();
-      constexpr int kCopies = 2 * HALVES * (kKeysPerTile / 4);
+      if (tile < ntiles) {
+        const uint32_t st = sKVa + (tile % NST) * 2 * SM::kTile;
 #pragma unroll
-      for (int c = lane; c < kCopies; c += 32) {
-        const int kv = c / (HALVES * 16), h = (c / 16) % HALVES, g4 = c % 16;
-        const int* rows = sIds + tile * kKeysPerTile + 4 * g4;
-        const uint32_t dst = sKVa + st * 2 * SM::kTile + kv * SM::kTile + h * SM::kHalfTile + g4 * 512;
-        tma_gather4(dst, kv ? &tmV : &tmK, h * 64, rows[0], rows[1], rows[2], rows[3], bar);
+        for (int u = 0; u < kKeysPerTile * 2 * PIECES / kAttnThreads; ++u) {
+          const int i = tid + u * kAttnThreads;
+          const int r = i / (2 * PIECES), rem = i % (2 * PIECES);
+          const int kv = rem / PIECES, c = rem % PIECES;
+          const int j = tile * kKeysPerTile + r;
+          const int s = j < n ? sIds[j] : -1;
+          const __nv_bfloat16* src = (kv ? Vb : Kb) + static_cast<int64_t>(s < 0 ? 0 : s) * D + c * 8;
+          cp_async16(st + kv * SM::kTile + kv_off<D>(r, c), src, s < 0 ? 0u : 16u);
+        }
       }
+      cp_async_commit();  // possibly empty: keeps one group per tile
     };
 #pragma unroll
     for (int t = 0; t < NST - 1; ++t) issue(t);
@@ -226,18 +191,17 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
 
     for (int tile = 0; tile < ntiles; ++tile) {
-      const uint32_t st = (gt + tile) % NST, ph = ((gt + tile) / NST) & 1;
-      mbar_wait(smem_u32(bars + st), ph, wait_limit_ns_device(), abort_flag);
-      __syncthreads();            // every warp is past tile - 1: its stage can be refilled
+      cp_async_wait<NST - 2>();   // this tile's copies (issued NST-1 tiles ago) are done
+      __syncthreads();            // ... for every thread; the oldest stage is free again
       issue(tile + NST - 1);
-      const uint32_t sK = sKVa + st * 2 * SM::kTile;
+      const uint32_t sK = sKVa + (tile % NST) * 2 * SM::kTile;
       const uint32_t sV = sK + SM::kTile;
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         uint32_t b[4];
         const int r = warp * 16 + (lane & 7) + (lane >> 4) * 8, c = kk * 2 + ((lane >> 3) & 1);
-        ldsm_x4(sK + kv_off(r, c), b);
+        ldsm_x4(sK + kv_off<D>(r, c), b);
         mma16816(s[0], qa[kk], b[0], b[1]);
         mma16816(s[1], qa[kk], b[2], b[3]);
       }
@@ -295,12 +259,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const __grid_constan
       for (int dt = 0; dt < D / 16; ++dt) {
         uint32_t b[4];
         const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = dt * 2 + (lane >> 4);
-        ldsm_x4_t(sV + kv_off(r, c), b);
+        ldsm_x4_t(sV + kv_off<D>(r, c), b);
         mma16816(o[2 * dt], pa, b[0], b[1]);
         mma16816(o[2 * dt + 1], pa, b[2], b[3]);
       }
     }
-    gt += ntiles;
+    cp_async_wait<0>();
     __syncthreads();  // all warps done with the tiles: the stage area becomes the merge area
 
     // ---- merge the four warps' partial states
@@ -379,28 +343,6 @@ __global__ void __launch_bounds__(D) combine_kernel(const float* part, int nspli
   O[(q * H + h) * D + col] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
 }
 
-// K or V [rows, D] BF16 as 2D tensor map for row gathers: one-row boxes of
-// 64 columns (128 bytes), 128-byte swizzle.
-bool make_row_map(CUtensorMap* m, const void* base, int D, int64_t rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess)
-      return false;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {64, 1};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p{a.Q, a.K, a.V, a.idx, a.ld_idx, a.nq, a.H, a.scale_log2, a.top_k, a.seq_start,
@@ -409,9 +351,6 @@ dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   static_assert(AttnSmem<D>::kStages * 2 * AttnSmem<D>::kTile >=
                     (4 * 16 * 2 + 4 * 16 * AttnSmem<D>::kMergeRow) * 4,
                 "merge area must fit in the tiles");
-  CUtensorMap tmK, tmV;
-  if (!make_row_map(&tmK, a.K, D, a.kv_rows) || !make_row_map(&tmV, a.V, D, a.kv_rows))
-    return DSA_ERR_CUDA;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return DSA_ERR_CUDA;
@@ -419,7 +358,7 @@ dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<D>, kAttnThreads, smem);
   const int64_t items = a.nq * a.nsplit;
   const int grid = static_cast<int>(std::min<int64_t>(items, std::max(1, per_sm) * num_sms()));
-  attn_kernel<D><<<grid, kAttnThreads, smem, stream>>>(tmK, tmV, p);
+  attn_kernel<D><<<grid, kAttnThreads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (a.nsplit > 1) {
     combine_kernel<D><<<static_cast<unsigned int>(a.nq * a.H), D, 0, stream>>>(a.part, a.nsplit,

@@ -109,52 +109,24 @@ __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
   return (f > 0.0f ? acc_bits : 0u) >> 16;  // non-negative float bits are monotone
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
+constexpr int kMiniRows = 8;                       // rows per sampled mini-tile
+constexpr int kMinisPerTile = kBN / kMiniRows;     // 32
 
-// Sample tile j of query tile qt: 256 key rows spread evenly over the keys
-// below the band [r0 - 128, r0 + 128) (stratified, so every region of the
-// prefix is represented), copied into the same 32-byte-swizzled K-major
-// layout the TMA path writes: row r, 16-byte chunk c of 32-byte slice b goes
-// to b * 8 KB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4).  All 32 lanes issue
-// cp.async copies and commit them as one group; sample_tile_done() completes
-// an older group.
-__device__ __forceinline__ void gather_sample_tile(const Params& p, const uint8_t* k_idx,
-                                                   int64_t qt, int j, int nt, uint32_t dst,
-                                                   int lane) {
-  const int pieces = 2 * p.nkb;                 // 16-byte pieces per row
-  const int rows_per_iter = 32 / pieces;        // nkb <= 16
-  const int rsub = lane / pieces, q = lane % pieces;
-  const int b = q >> 1, c = q & 1;
-  const uint64_t span = static_cast<uint64_t>(qt * kBM - 128);  // keys [0, span) below the band
-  const uint64_t ns = static_cast<uint64_t>(nt) * kBN;           // ns <= span
-  const uint64_t step16 = (span << 16) / ns;                     // span / ns in 48.16 fixed point
-  const int64_t row_bytes = static_cast<int64_t>(p.nkb) * 32;
-  if (rsub < rows_per_iter) {
-    for (int r = rsub; r < kBN; r += rows_per_iter) {
-      // key = floor(i * span / ns) up to the fixed-point truncation: < span, nondecreasing
-      const int64_t key = static_cast<int64_t>((static_cast<uint64_t>(j * kBN + r) * step16) >> 16);
-      cp_async16(dst + b * kTileB + r * 32 + ((c ^ ((r >> 2) & 1)) << 4),
-                 k_idx + key * row_bytes + q * 16);
-    }
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// Waits until at most `pending` gather groups of this lane are in flight, then
-// makes the landed rows visible to the tensor core (async proxy) for the warp.
-template <int PENDING>
-__device__ __forceinline__ void sample_tile_done() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(PENDING) : "memory");
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncwarp();
+// First key of mini-tile i (0 .. nt*32-1) of query tile qt: the mini-tiles
+// are spread evenly over the keys below the band [r0 - 128, r0 + 128), so
+// every region of the prefix is represented (a stratified sample), and each
+// stays inside it.
+__device__ __forceinline__ int mini_tile_row(int64_t qt, int i, int nt) {
+  const uint64_t span = static_cast<uint64_t>(qt * kBM - 128);     // keys [0, span)
+  const uint64_t nmini = static_cast<uint64_t>(nt) * kMinisPerTile;
+  const uint64_t room = span - kMiniRows;                          // span >= 256 * nt
+  return static_cast<int>((static_cast<uint64_t>(i) * room) / (nmini - 1 > 0 ? nmini - 1 : 1));
 }
 
 template <int ESIZE>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const Params p) {
+                   const __grid_constant__ CUtensorMap tmK8, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -204,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Lane 0 issues the TMA copies and barrier operations.  In sample mode the
-    // whole warp gathers the sampled key rows with cp.async instead.
+    // whole warp issues them, one 8-row mini-tile per lane.
     const bool gather = p.mode == kModeSample;
     if (gather || lane == 0) {
       uint32_t it = 0, item_it = 0;
@@ -239,23 +211,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < p.nkb; ++b)
               tma_load_2d(dst + b * kTileB, &tmK, b * (32 / ESIZE), kt * kBN, bar(FULL + s));
           } else {
-            // Two tiles in flight: issue tile j, then publish tile j-1.  With a
-            // single stage, tile j's slot frees only after tile j-1 is consumed,
-            // so publish each tile right away.
-            gather_sample_tile(p, static_cast<const uint8_t*>(p.k_idx), qt, j, nt, dst, lane);
-            if (S == 1) {
-              sample_tile_done<0>();
-              if (lane == 0) mbar_arrive(bar(FULL + s));
-            } else if (j > 0) {
-              sample_tile_done<1>();
-              if (lane == 0) mbar_arrive(bar(FULL + (it - 1) % S));
-            }
+            // 32 mini-tiles of 8 consecutive keys; each lane loads one mini-tile
+            // (all 32-byte slices) into rows 8*lane .. 8*lane+7 of the stage.
+            if (lane == 0) mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
+            __syncwarp();
+            const int y = mini_tile_row(qt, j * kMinisPerTile + lane, nt);
+            for (int b = 0; b < p.nkb; ++b)
+              tma_load_2d(dst + b * kTileB + lane * kMiniRows * 32, &tmK8, b * (32 / ESIZE), y,
+                          bar(FULL + s));
           }
           ++it;
-        }
-        if (gather) {  // publish the item's last tile (or drain after an abort)
-          sample_tile_done<0>();
-          if (ok && S > 1 && lane == 0) mbar_arrive(bar(FULL + (it - 1) % S));
         }
       }
       if (lane == 0) {
@@ -592,9 +557,10 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   // At least 116 KB so two CTAs never share an SM (each holds all 512 TMEM columns).
   const size_t smem = std::max<size_t>(p.off_bar + kMiscBytes + 1024, 116 * 1024);
 
-  CUtensorMap tmQ, tmK;
+  CUtensorMap tmQ, tmK, tmK8;
   if (!make_map(&tmQ, a.q_idx, a.esize, a.d, a.Lq, kBM) ||
-      !make_map(&tmK, a.k_idx, a.esize, a.d, a.Lk, kBN))
+      !make_map(&tmK, a.k_idx, a.esize, a.d, a.Lk, kBN) ||
+      !make_map(&tmK8, a.k_idx, a.esize, a.d, a.Lk, kMiniRows))
     return DSA_ERR_CUDA;
 
   const int grid = std::max(1, std::min(p.n_items, num_sms()));
@@ -602,11 +568,11 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   if (a.esize == 1) {
     e = cudaFuncSetAttribute(indexer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-    if (e == cudaSuccess) indexer_kernel<1><<<grid, kThreads, smem, stream>>>(tmQ, tmK, p);
+    if (e == cudaSuccess) indexer_kernel<1><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmK8, p);
   } else {
     e = cudaFuncSetAttribute(indexer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-    if (e == cudaSuccess) indexer_kernel<2><<<grid, kThreads, smem, stream>>>(tmQ, tmK, p);
+    if (e == cudaSuccess) indexer_kernel<2><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmK8, p);
   }
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
