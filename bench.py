@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--workload", default=PREFILL,
                     choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k"],
                     help="prefill workload of a step (smaller ones for profiling)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="decode only the first B sequences of the batch (profiling)")
     return ap.parse_args()
 
 
@@ -368,6 +370,9 @@ def main():
         wd = synth.WORKLOADS[DECODE]
         del ws
         torch.cuda.empty_cache()
+        if args.decode_batch:
+            import dataclasses
+            wd = dataclasses.replace(wd, B=args.decode_batch)
         xd = synth.decode_inputs_torch(wd, seed=seed, device=dev)
         lengths = xd["lengths"]
         wsd = torch.empty(dsa.dsa_decode_workspace_size(wd.B, int(lengths.sum()), wd.d_idx, 0, wd.H, wd.D,
