@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sort.cuh"
 
 namespace dsa {
 
@@ -30,7 +31,9 @@ constexpr int kScanThreads = 256;
 constexpr int kScanRowsPerCta = 4096;
 constexpr int kHistBins = 2048;           // score bits 30..20 (scores are >= +0)
 constexpr int kSelThreads = 1024;
-constexpr int kSmemKeys = 12288;          // candidates held in shared memory
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelSlots = 8;
+constexpr int kSmemKeys = kSelWarps * 32 * kSelSlots;   // 8192 candidates held in shared memory
 
 __device__ __forceinline__ unsigned long long score_key(float sc, uint32_t s) {
   return (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xFFFFFFFFu - s);
@@ -148,6 +151,85 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
     if (hist[i]) atomicAdd(&p.hist[static_cast<int64_t>(b) * kHistBins + i], hist[i]);
 }
 
+// Coalesced variant for rows of LPR x 16 bytes (LPR a power of two): LPR
+// lanes share a row, each holding its 16-byte slice of the query in
+// registers; a warp load covers 32 / LPR consecutive rows, eight loads are in
+// flight per lane, and log2(LPR) shuffles finish each row's dot product.
+template <int ESIZE, int LPR>
+__global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const ScanParams p) {
+  constexpr int RPL = 32 / LPR;                 // rows per warp load
+  constexpr int U = 8;                          // loads in flight per lane
+  constexpr int VALS = 16 / ESIZE;              // index values per 16-byte slice
+  __shared__ unsigned int hist[kHistBins];
+  if (*p.invalid) return;
+  const int b = blockIdx.y;
+  const int64_t base = p.seq_start[b];
+  const int64_t len = p.seq_start[b + 1] - base;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kScanRowsPerCta;
+  if (c0 >= len) return;
+  const int64_t c1 = min64(len, c0 + kScanRowsPerCta);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane % LPR, rsub = lane / LPR;
+  float qv[VALS];
+#pragma unroll
+  for (int i = 0; i < VALS; ++i) {
+    const int j = sub * VALS + i;
+    if (ESIZE == 1) {
+      const __nv_fp8_storage_t v = static_cast<const __nv_fp8_storage_t*>(p.q_idx)[b * p.d + j];
+      qv[i] = __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)));
+    } else {
+      qv[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q_idx)[b * p.d + j]);
+    }
+  }
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const uint8_t* rows = static_cast<const uint8_t*>(p.k_idx) + base * (LPR * 16);
+  for (int64_t r0 = c0 + warp * RPL * U; r0 < c1; r0 += (kScanThreads / 32) * RPL * U) {
+    uint4 w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t r = r0 + u * RPL + rsub;
+      w[u] = r < c1 ? __ldg(reinterpret_cast<const uint4*>(rows + r * (LPR * 16) + sub * 16))
+                    : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+      float acc = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (ESIZE == 1) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const __nv_fp8x2_storage_t pair =
+                static_cast<__nv_fp8x2_storage_t>((words[k] >> (16 * h)) & 0xFFFFu);
+            const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
+            acc = fmaf(qv[4 * k + 2 * h], f.x, acc);
+            acc = fmaf(qv[4 * k + 2 * h + 1], f.y, acc);
+          }
+        } else {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&words[k]));
+          acc = fmaf(qv[2 * k], f.x, acc);
+          acc = fmaf(qv[2 * k + 1], f.y, acc);
+        }
+      }
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+      const int64_t r = r0 + u * RPL + rsub;
+      if (sub == 0 && r < c1) {
+        float sc = __fmul_rn(acc, p.scale);
+        sc = sc > 0.0f ? sc : 0.0f;
+        p.scores[base + r] = sc;
+        const uint32_t bin = __float_as_uint(sc) >> 20;
+        if (bin) atomicAdd(&hist[bin], 1u);  // zero scores are recovered by the select
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+    if (hist[i]) atomicAdd(&p.hist[static_cast<int64_t>(b) * kHistBins + i], hist[i]);
+}
+
 // ---- select ------------------------------------------------------------------
 
 __device__ __forceinline__ void find_from_top_256(const unsigned int* hist, int R, int* out) {
@@ -231,22 +313,26 @@ struct DSelParams {
 
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelParams p) {
   extern __shared__ unsigned long long ds_smem[];
-  unsigned long long* keys = ds_smem;                       // [kSmemKeys]
-  unsigned long long* sel = keys + kSmemKeys;               // [2048]
-  unsigned int* h256 = reinterpret_cast<unsigned int*>(sel + DSA_MAX_TOP_K);
-  int* sh = reinterpret_cast<int*>(h256 + 256);             // [8]
+  unsigned long long* bufA = ds_smem;                              // [kSmemKeys]
+  unsigned long long* bufB = bufA + kSmemKeys;                     // [kSmemKeys]
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(bufB + kSmemKeys);   // [warps][256]
+  uint32_t* dbase = cnt + kSelWarps * 256;                         // [256]
+  uint32_t* wsum = dbase + 256;                                    // [warps]
+  int* sh = reinterpret_cast<int*>(wsum + kSelWarps);              // [8]
+  unsigned int* h256 = dbase;                                      // fallback path histogram
   if (*p.invalid) return;
   const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t base = p.seq_start[b];
   const int n = static_cast<int>(p.seq_start[b + 1] - base);
   const int m = min(p.top_k, n);
   const float* sc = p.scores + base;
   const unsigned int* hist = p.hist + static_cast<int64_t>(b) * kHistBins;
+  int32_t* out = p.indices + static_cast<int64_t>(b) * p.top_k;
 
   // Bin of the m-th best score (bins scanned from the top by warp 0).  Bin 0
   // (score +0) is not counted by the scan: every key not in a higher bin.
   if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
     unsigned int local = 0;
     for (int i = 0; i < kHistBins / 32; ++i) {
       const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
@@ -273,18 +359,84 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
         }
       }
     }
+    if (lane == 0) {
+      sh[2] = 0;            // compacted so far
+      sh[3] = 0;            // OR of score words
+      sh[4] = -1;           // AND of score words
+    }
   }
   __syncthreads();
   const uint32_t bin = static_cast<uint32_t>(sh[0]);
   const int ncand = sh[1];
-  __syncthreads();
 
-  unsigned long long* cand;
   if (ncand <= kSmemKeys) {
-    cand = keys;
-  } else {
-    cand = p.scratch + base;
+    // Stable compaction of the candidates (score bin >= bin) in index order.
+    uint32_t o_or = 0u, o_and = 0xFFFFFFFFu;
+    for (int s0 = 0; s0 < n; s0 += kSelThreads * 4) {
+      const int s = s0 + threadIdx.x * 4;
+      float v[4];
+      uint32_t flags = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[k] = s + k < n ? sc[s + k] : 0.0f;
+        if (s + k < n && (__float_as_uint(v[k]) >> 20) >= bin) flags |= 1u << k;
+      }
+      const uint32_t c = __popc(flags);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t x = wsum[lane];
+        uint32_t wi = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+          if (lane >= o) wi += y;
+        }
+        wsum[lane] = wi - x;        // exclusive warp offsets
+        if (lane == 31) sh[5] = static_cast<int>(wi);
+      }
+      __syncthreads();
+      int pos = sh[2] + static_cast<int>(wsum[warp] + incl - c);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (flags & (1u << k)) {
+          const uint32_t bits = __float_as_uint(v[k]);
+          o_or |= bits;
+          o_and &= bits;
+          if (pos < kSmemKeys) bufA[pos] = score_key(v[k], static_cast<uint32_t>(s + k));
+          ++pos;
+        }
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) sh[2] += sh[5];
+      __syncthreads();
+    }
+    o_or = __reduce_or_sync(0xFFFFFFFFu, o_or);
+    o_and = __reduce_and_sync(0xFFFFFFFFu, o_and);
+    if (lane == 0) {
+      atomicOr(reinterpret_cast<unsigned int*>(&sh[3]), o_or);
+      atomicAnd(reinterpret_cast<unsigned int*>(&sh[4]), o_and);
+    }
+    __syncthreads();
+    const int nc = min(sh[2], kSmemKeys);
+    const uint32_t vary = static_cast<uint32_t>(sh[3]) ^ static_cast<uint32_t>(sh[4]);
+    const unsigned long long* cur =
+        stable_sort_by_score<kSelWarps, kSelSlots>(bufA, bufB, nc, vary, cnt, dbase);
+    for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
+      out[i] = i < m && i < nc ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(cur[i]))
+                               : -1;
+    return;
   }
+
+  // Many candidates (wide ties): compact into the global scratch row, select
+  // the m-th key by radix passes there, then sort the m winners.
+  unsigned long long* cand = p.scratch + base;
   if (threadIdx.x == 0) sh[2] = 0;
   __syncthreads();
   for (int s = threadIdx.x; s < n; s += blockDim.x) {
@@ -296,6 +448,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   }
   __syncthreads();
   const unsigned long long kth = ncand > m ? radix_select(cand, ncand, m, h256, sh) : 0ull;
+  unsigned long long* sel = bufA;
   if (threadIdx.x == 0) sh[3] = 0;
   __syncthreads();
   for (int i = threadIdx.x; i < ncand; i += blockDim.x) {
@@ -311,8 +464,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   for (int i = m + threadIdx.x; i < P; i += blockDim.x) sel[i] = 0ull;
   bitonic_desc(sel, P);
   for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
-    p.indices[static_cast<int64_t>(b) * p.top_k + i] =
-        i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
+    out[i] = i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
 }
 
 }  // namespace
@@ -324,14 +476,26 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
   ScanParams sp{a.k_idx, a.q_idx, a.d, a.seq_start, a.scale, a.scores, a.hist, a.invalid};
   const dim3 grid(static_cast<unsigned int>((a.max_len + kScanRowsPerCta - 1) / kScanRowsPerCta),
                   static_cast<unsigned int>(a.B));
-  if (a.esize == 1)
+  const int lpr = a.d * a.esize / 16;  // 16-byte slices per index row
+  if (a.esize == 1 && lpr == 8)
+    decode_scan_rows_kernel<1, 8><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (a.esize == 1 && lpr == 4)
+    decode_scan_rows_kernel<1, 4><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (a.esize == 1 && lpr == 16)
+    decode_scan_rows_kernel<1, 16><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (a.esize == 2 && lpr == 8)
+    decode_scan_rows_kernel<2, 8><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (a.esize == 2 && lpr == 16)
+    decode_scan_rows_kernel<2, 16><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (a.esize == 1)
     decode_scan_kernel<1><<<grid, kScanThreads, 0, stream>>>(sp);
   else
     decode_scan_kernel<2><<<grid, kScanThreads, 0, stream>>>(sp);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
 
   DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid};
-  const size_t smem = static_cast<size_t>(kSmemKeys + DSA_MAX_TOP_K) * 8 + 256 * 4 + 32;
+  const size_t smem = static_cast<size_t>(2 * kSmemKeys) * 8 +
+                      (kSelWarps * 256 + 256 + kSelWarps + 8) * 4;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "sort.cuh"
 
 namespace dsa {
 
@@ -174,74 +175,6 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
   }
 }
 
-// Stable pass: out = in ordered by byte (key >> shift) & 255, descending.
-__device__ void radix_pass_desc(const unsigned long long* in, unsigned long long* out, int n,
-                                int shift, uint32_t* cnt /*[warps][256]*/, uint32_t* base /*[256]*/) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = (n + kSortWarps * 32 - 1) / (kSortWarps * 32) * 32;  // items per warp
-  const int slots = chunk / 32;
-  uint32_t* wc = cnt + warp * 256;
-  for (int d = lane; d < 256; d += 32) wc[d] = 0;
-  __syncwarp();
-  const uint32_t lt = (1u << lane) - 1u;
-  unsigned long long v[kSortMaxSlots];
-  uint32_t dg[kSortMaxSlots], rk[kSortMaxSlots];
-#pragma unroll
-  for (int j = 0; j < kSortMaxSlots; ++j) {
-    if (j < slots) {
-      const int i = warp * chunk + j * 32 + lane;
-      const bool ok = i < n;
-      v[j] = ok ? in[i] : 0ull;
-      const uint32_t d = ok ? 255u - static_cast<uint32_t>((v[j] >> shift) & 255u) : 256u;
-      dg[j] = d;
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
-      const uint32_t before = ok ? wc[d] : 0u;
-      rk[j] = before + __popc(peers & lt);
-      __syncwarp();
-      if (ok && lane == __ffs(peers) - 1) wc[d] = before + __popc(peers);
-      __syncwarp();
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < 256) {  // per digit: warp-exclusive prefix, digit total
-    const int d = threadIdx.x;
-    uint32_t run = 0;
-    for (int w = 0; w < kSortWarps; ++w) {
-      const uint32_t c = cnt[w * 256 + d];
-      cnt[w * 256 + d] = run;
-      run += c;
-    }
-    base[d] = run;
-  }
-  __syncthreads();
-  if (threadIdx.x < 32) {  // exclusive scan of the 256 digit totals
-    uint32_t loc[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      loc[q] = base[lane * 8 + q];
-      sum += loc[q];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    uint32_t ex = incl - sum;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      base[lane * 8 + q] = ex;
-      ex += loc[q];
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int j = 0; j < kSortMaxSlots; ++j) {
-    if (j < slots && dg[j] < 256u) out[base[dg[j]] + cnt[warp * 256 + dg[j]] + rk[j]] = v[j];
-  }
-  __syncthreads();
-}
-
 struct SelParams {
   int64_t L;
   int top_k, cap;
@@ -310,7 +243,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     unsigned long long* nxt = bufA;
     for (int byte = 0; byte < 4; ++byte) {
       if ((vary >> (8 * byte)) & 255u) {
-        radix_pass_desc(cur, nxt, n, 32 + 8 * byte, cnt, base);
+        radix_pass_desc<kSortWarps, kSortMaxSlots>(cur, nxt, n, 32 + 8 * byte, cnt, base);
         unsigned long long* tmp = cur;
         cur = nxt;
         nxt = tmp;

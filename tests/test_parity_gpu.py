@@ -257,6 +257,19 @@ def test_decode_small_top_k(dsa):
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
 
 
+@pytest.mark.parametrize("idx_dtype,d,top_k", [("fp8", 64, 300), ("fp8", 256, 512), ("bf16", 128, 256),
+                                               ("bf16", 160, 128)])
+def test_decode_index_formats(dsa, idx_dtype, d, top_k):
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["decode_64x128k"], d_idx=d, idx_dtype=idx_dtype)
+    lens = np.array([7, 513, 4100, 20000], dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    idx, O = run_decode(dsa, xd, top_k)
+    ri, ro = oracle.decode(xd, idx_dtype, top_k)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
 def test_decode_full_workload(dsa):
     w = synth.WORKLOADS["decode_64x128k"]
     xd = host_copy(synth.decode_inputs_torch(w, device="cuda"))
