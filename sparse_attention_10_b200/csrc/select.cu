@@ -153,9 +153,11 @@ __device__ __forceinline__ uint32_t key_index(unsigned long long k) {
   return 0xFFFFFFFFu - static_cast<uint32_t>(k);
 }
 
-// Merge two ascending-index runs a[0, na) and b[0, nb) into out (merge path).
+// Merge two ascending-index runs a[0, na) and b[0, nb) (64-bit candidate
+// keys) into one ascending-index run, written as score words `sc` and key
+// indices `ix` (merge path: each thread finds its split by binary search).
 __device__ void merge_by_index(const unsigned long long* a, int na, const unsigned long long* b,
-                               int nb, unsigned long long* out) {
+                               int nb, uint32_t* sc, uint32_t* ix) {
   const int n = na + nb;
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int p0 = min(n, static_cast<int>(threadIdx.x) * per), p1 = min(n, p0 + per);
@@ -171,7 +173,9 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
   int i = lo, j = p0 - lo;
   for (int p = p0; p < p1; ++p) {
     const bool take_a = j >= nb || (i < na && key_index(a[i]) < key_index(b[j]));
-    out[p] = take_a ? a[i++] : b[j++];
+    const unsigned long long k = take_a ? a[i++] : b[j++];
+    sc[p] = static_cast<uint32_t>(k >> 32);
+    ix[p] = key_index(k);
   }
 }
 
@@ -188,11 +192,17 @@ struct SelParams {
 
 __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long sel_smem[];
-  unsigned long long* bufA = sel_smem;                          // [kSortCap]
-  unsigned long long* bufB = bufA + kSortCap;                   // [kSortCap]
-  uint32_t* cnt = reinterpret_cast<uint32_t*>(bufB + kSortCap); // [warps][256] (also the bitmap)
-  uint32_t* base = cnt + kSortWarps * 256;                      // [256]
-  uint32_t* misc = base + 256;                                  // [8]
+  // raw: the row's two candidate lists (64-bit keys); after the merge the same
+  // bytes hold the second score buffer and both position buffers.
+  unsigned long long* raw = sel_smem;                                    // [kSortCap]
+  uint32_t* sc1 = reinterpret_cast<uint32_t*>(raw);                      // [kSortCap]
+  uint16_t* ps0 = reinterpret_cast<uint16_t*>(sc1 + kSortCap);           // [kSortCap]
+  uint16_t* ps1 = ps0 + kSortCap;                                        // [kSortCap]
+  uint32_t* sc0 = reinterpret_cast<uint32_t*>(raw + kSortCap);           // [kSortCap]
+  uint32_t* ix = sc0 + kSortCap;                                         // [kSortCap]
+  uint32_t* cnt = ix + kSortCap;                                         // [warps][256] / bitmap
+  uint32_t* base = cnt + kSortWarps * 256;                               // [256]
+  uint32_t* misc = base + 256;                                           // [8]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
@@ -216,14 +226,14 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
     const unsigned long long* c1 = c0 + p.cap;
-    for (int i = threadIdx.x; i < n0; i += blockDim.x) bufA[i] = c0[i];
-    for (int i = threadIdx.x; i < n1; i += blockDim.x) bufA[n0 + i] = c1[i];
+    for (int i = threadIdx.x; i < n0; i += blockDim.x) raw[i] = c0[i];
+    for (int i = threadIdx.x; i < n1; i += blockDim.x) raw[n0 + i] = c1[i];
     __syncthreads();
-    merge_by_index(bufA, n0, bufA + n0, n1, bufB);
+    merge_by_index(raw, n0, raw + n0, n1, sc0, ix);
     __syncthreads();
     uint32_t o = 0u, a = 0xFFFFFFFFu, pos = 0u;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t hi = static_cast<uint32_t>(bufB[i] >> 32);
+      const uint32_t hi = sc0[i];
       o |= hi;
       a &= hi;
       pos += hi != 0u;
@@ -239,20 +249,13 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     __syncthreads();
     const uint32_t vary = misc[0] ^ misc[1];
     const int npos = static_cast<int>(misc[2]);
-    unsigned long long* cur = bufB;
-    unsigned long long* nxt = bufA;
-    for (int byte = 0; byte < 4; ++byte) {
-      if ((vary >> (8 * byte)) & 255u) {
-        radix_pass_desc<kSortWarps, kSortMaxSlots>(cur, nxt, n, 32 + 8 * byte, cnt, base);
-        unsigned long long* tmp = cur;
-        cur = nxt;
-        nxt = tmp;
-      }
-    }
+    uint32_t* ks = sc0;
+    uint16_t* ps = nullptr;
+    stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary, cnt, base);
     int32_t* out = p.indices + t * p.top_k;
     if (!zero_mode || npos >= m) {
       for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
-        out[i] = i < m ? static_cast<int32_t>(key_index(cur[i])) : -1;
+        out[i] = i < m ? static_cast<int32_t>(ix[ps ? ps[i] : i]) : -1;
     } else {
       // Every positive score is a candidate; the rest of the row ranks the
       // zero scores by ascending key index.  Within keys [0, R) there are at
@@ -263,12 +266,11 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
       for (int wd = threadIdx.x; wd < words; wd += blockDim.x) bm[wd] = 0u;
       __syncthreads();
       for (int i = threadIdx.x; i < npos; i += blockDim.x) {
-        const uint32_t s = key_index(cur[i]);
-        if (s < static_cast<uint32_t>(R)) atomicOr(&bm[s >> 5], 1u << (s & 31));
-        out[i] = static_cast<int32_t>(s);
+        const uint32_t sidx = ix[ps ? ps[i] : i];
+        if (sidx < static_cast<uint32_t>(R)) atomicOr(&bm[sidx >> 5], 1u << (sidx & 31));
+        out[i] = static_cast<int32_t>(sidx);
       }
       __syncthreads();
-      // zero count per word, exclusive scan over words (words <= 128)
       uint32_t z = 0u;
       if (threadIdx.x < words) {
         const int wd = threadIdx.x;
@@ -294,9 +296,9 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
         const uint32_t valid = (wd * 32 + 32 <= R) ? 0xFFFFFFFFu : ((1u << (R - wd * 32)) - 1u);
         uint32_t zeros = ~bm[wd] & valid;
         while (zeros) {
-          const int b = __ffs(zeros) - 1;
+          const int bit = __ffs(zeros) - 1;
           zeros &= zeros - 1u;
-          if (rank < static_cast<uint32_t>(m - npos)) out[npos + rank] = wd * 32 + b;
+          if (rank < static_cast<uint32_t>(m - npos)) out[npos + rank] = wd * 32 + bit;
           ++rank;
         }
       }
@@ -410,7 +412,7 @@ dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
   if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
   SelParams p{a.L, a.top_k, a.cap, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
-  const size_t smem = 2 * static_cast<size_t>(kSortCap) * 8 + (kSortWarps * 256 + 256 + 8) * 4;
+  const size_t smem = static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return DSA_ERR_CUDA;

@@ -102,3 +102,116 @@ __device__ unsigned long long* stable_sort_by_score(unsigned long long* a, unsig
 }
 
 }  // namespace dsa
+
+namespace dsa {
+
+// Stable pass on 32-bit score words with 16-bit payloads (positions):
+// (kout, pout) = (kin, pin) ordered by byte SHIFT/8 of the key, DESCENDING,
+// equal bytes in input order.  pin == nullptr means the identity payload.
+// Same warp/slot/lane ownership and atomic-free ranking as radix_pass_desc.
+template <int WARPS, int SLOTS, int SHIFT>
+__device__ void radix_pass32_desc(const uint32_t* kin, const uint16_t* pin, uint32_t* kout,
+                                  uint16_t* pout, int n, uint32_t* cnt, uint32_t* base) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = (n + WARPS * 32 - 1) / (WARPS * 32) * 32;  // items per warp
+  const int slots = chunk / 32;
+  uint32_t* wc = cnt + warp * 256;
+  for (int d = lane; d < 256; d += 32) wc[d] = 0;
+  __syncwarp();
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t dr[SLOTS];  // digit (bits 16..24, 256 = no item) | rank in warp (bits 0..15)
+#pragma unroll
+  for (int j = 0; j < SLOTS; ++j) {
+    if (j < slots) {
+      const int i = warp * chunk + j * 32 + lane;
+      const bool ok = i < n;
+      const uint32_t d = ok ? 255u - ((kin[i] >> SHIFT) & 255u) : 256u;
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
+      const uint32_t before = ok ? wc[d] : 0u;
+      dr[j] = (d << 16) | (before + __popc(peers & lt));
+      __syncwarp();
+      if (ok && lane == __ffs(peers) - 1) wc[d] = before + __popc(peers);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < 256) {  // per digit: warp-exclusive prefix, digit total
+    const int d = threadIdx.x;
+    uint32_t run = 0;
+#pragma unroll 4
+    for (int w = 0; w < WARPS; ++w) {
+      const uint32_t c = cnt[w * 256 + d];
+      cnt[w * 256 + d] = run;
+      run += c;
+    }
+    base[d] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // exclusive scan of the 256 digit totals
+    uint32_t loc[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      loc[q] = base[lane * 8 + q];
+      sum += loc[q];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t ex = incl - sum;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      base[lane * 8 + q] = ex;
+      ex += loc[q];
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < SLOTS; ++j) {
+    if (j < slots) {
+      const uint32_t d = dr[j] >> 16;
+      if (d < 256u) {
+        const int i = warp * chunk + j * 32 + lane;
+        const uint32_t pos = base[d] + cnt[warp * 256 + d] + (dr[j] & 0xFFFFu);
+        kout[pos] = kin[i];
+        pout[pos] = pin ? pin[i] : static_cast<uint16_t>(i);
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Stable sort of (score word, position) pairs, descending by score, one pass
+// per differing score byte.  Returns through *k / *p the buffers holding the
+// result; p0 == nullptr on entry means positions 0..n-1.
+template <int WARPS, int SLOTS>
+__device__ void stable_sort32_by_score(uint32_t** k, uint16_t** p, uint32_t* k_alt,
+                                       uint16_t* p_alt, uint16_t* p_first, int n, uint32_t vary,
+                                       uint32_t* cnt, uint32_t* base) {
+  uint32_t* kc = *k;
+  uint16_t* pc = nullptr;             // identity until the first pass
+  uint32_t* kn = k_alt;
+  uint16_t* pn = p_first;
+  uint16_t* spare = p_alt;
+#define DSA_PASS(SH)                                                                  \
+  if ((vary >> SH) & 255u) {                                                          \
+    radix_pass32_desc<WARPS, SLOTS, SH>(kc, pc, kn, pn, n, cnt, base);                \
+    uint32_t* tk = kc;                                                                \
+    kc = kn;                                                                          \
+    kn = tk;                                                                          \
+    uint16_t* tp = pc ? pc : spare;                                                   \
+    pc = pn;                                                                          \
+    pn = tp;                                                                          \
+  }
+  DSA_PASS(0)
+  DSA_PASS(8)
+  DSA_PASS(16)
+  DSA_PASS(24)
+#undef DSA_PASS
+  *k = kc;
+  *p = pc;  // nullptr: no pass ran, order is the input order
+}
+
+}  // namespace dsa
