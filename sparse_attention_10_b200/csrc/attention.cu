@@ -145,14 +145,19 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     const __nv_bfloat16* Vb = p.V + row_base * D;
 
     // Q rows (heads >= H are zero) and this item's key list, clamped.
+    // (asynchronous copies: every row of Q and the whole key list in flight at once)
     for (int i = tid; i < 16 * PIECES; i += kAttnThreads) {
       const int r = i / PIECES, c = i % PIECES;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < p.H) v = *reinterpret_cast<const uint4*>(p.Q + (q * p.H + r) * D + c * 8);
-      *reinterpret_cast<uint4*>(sQ + r * SM::kRowQ + c * 16) = v;
+      cp_async16(smem_u32(sQ + r * SM::kRowQ + c * 16), p.Q + (q * p.H + min(r, p.H - 1)) * D + c * 8,
+                 r < p.H ? 16u : 0u);
     }
+    for (int i = tid; i < n; i += kAttnThreads)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sIds + i)), "l"(ids + i)
+                   : "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
     for (int i = tid; i < n; i += kAttnThreads) {
-      const int s = ids[i];
+      const int s = sIds[i];
       sIds[i] = (s >= 0 && s < row_limit) ? s : -1;
     }
     __syncthreads();

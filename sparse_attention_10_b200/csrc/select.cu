@@ -226,8 +226,13 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
     const unsigned long long* c1 = c0 + p.cap;
-    for (int i = threadIdx.x; i < n0; i += blockDim.x) raw[i] = c0[i];
-    for (int i = threadIdx.x; i < n1; i += blockDim.x) raw[n0 + i] = c1[i];
+    // Both lists in flight at once (8-byte asynchronous copies), one wait.
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long* src = i < n0 ? c0 + i : c1 + (i - n0);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(raw + i)), "l"(src)
+                   : "memory");
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     merge_by_index(raw, n0, raw + n0, n1, sc0, ix);
     __syncthreads();
