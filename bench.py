@@ -72,6 +72,40 @@ def peaks():
     return p
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def source_sha256(rel_path: str) -> str:
+    import hashlib
+    with open(os.path.join(ROOT, rel_path), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def profiled_traffic(kernel: str, workload: str, source: str):
+    """DRAM bytes per launch from profiles/<kernel>_<workload>.md, or None when the
+    summary is missing or the kernel source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        fields = {}
+        for line in open(path):
+            if line.startswith("- ") and ":" in line:
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+        if fields.get("source_sha256") != source_sha256(source):
+            return None
+        return float(fields["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -258,11 +292,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     w = synth.WORKLOADS[args.workload]
     seed = synth.SEED + rank              # every rank runs its own sequence
@@ -284,6 +314,7 @@ def main():
     if dsa.dsa_sync_status(stream) != 0:
         raise RuntimeError("device-side error during warm-up")
     stats = dsa.dsa_last_stats(ws)
+    work_cand = 8.0 * stats["candidates"]
 
     # --- timed region: K prefill steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -310,6 +341,7 @@ def main():
     stages = dsa.dsa_stage_times()
     launches_per_step = sum(v[1] for v in stages.values()) / args.steps
     work = prefill_work(w)
+    work["cand_bytes"] = work_cand
     pk = peaks()
     st_ms = {k_: v[0] / args.steps for k_, v in stages.items() if v[1] > 0}
     idx_ms = st_ms.get("indexer_filter", float("nan"))
@@ -318,15 +350,29 @@ def main():
     gather_gbs = work["gather_bytes"] / (att_ms / 1000.0) / 1e9
     dominant = max(("indexer_filter", "attention", "select", "indexer_sample", "threshold"),
                    key=lambda s: st_ms.get(s, 0.0))
+    # A contraction takes the peak of its own dtype: BF16 measured; FP8 = 2 x BF16 measured
+    # (the nominal dense FP8:BF16 ratio).  Sustained figures: the kernels run inside a long step.
+    idx_peak = pk["bf16_tflops_sustained"] * (2.0 if w.idx_dtype == "fp8" else 1.0)
+    fp8_peak = 2.0 * pk["bf16_tflops_sustained"]
+    indexer = {"tflops": indexer_tflops, "dtype": w.idx_dtype, "peak_own_dtype": idx_peak,
+               "frac_own_dtype": indexer_tflops / idx_peak, "frac_fp8_peak": indexer_tflops / fp8_peak,
+               "flops_per_launch": work["indexer_flops"], "ms": idx_ms}
     if dominant.startswith("indexer"):
         flops = work["indexer_flops"] if dominant == "indexer_filter" else float("nan")
         ach = flops / (st_ms[dominant] / 1000.0) / 1e12
-        roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops_sustained"], "traffic": None}
+        roof = {"kernel": "indexer_kernel", "bound": "tensor", "achieved": ach, "peak": idx_peak,
+                "unit": "TFLOP/s", "frac": ach / idx_peak,
+                "traffic": profiled_traffic("indexer_kernel", w.name, "sparse_attention_10_b200/csrc/indexer.cu")}
+    elif dominant == "attention":
+        ach = work["attn_bytes"] / (st_ms["attention"] / 1000.0) / 1e9
+        roof = {"kernel": "attn_kernel", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "bytes_per_launch": work["attn_bytes"],
+                "traffic": profiled_traffic("attn_kernel", w.name, "sparse_attention_10_b200/csrc/attention.cu")}
     else:
-        ach = work["attn_bytes"] / (st_ms["attention"] / 1000.0) / 1e9 if dominant == "attention" else float("nan")
-        roof = {"kernel": dominant, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "traffic": None}
+        ach = (work["cand_bytes"] + 4.0 * w.L * w.top_k) / (st_ms[dominant] / 1000.0) / 1e9
+        roof = {"kernel": "select_kernel", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"],
+                "traffic": profiled_traffic("select_kernel", w.name, "sparse_attention_10_b200/csrc/select.cu")}
     roof["peak_source"] = pk["source"]
 
     # --- end to end through the public API with host buffers
@@ -434,7 +480,7 @@ def main():
                                    f"Q [L,{w.H},{w.D}], K/V [L,{w.D}] bf16 N(0,1), top_k={w.top_k}",
                        "parallelism": f"{world} independent sequences (one per GPU)",
                        "l2": "inputs larger than L2 (~9 GB touched per step vs 126 MB L2)"},
-            "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs,
+            "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs, "indexer": indexer,
             "stage_ms": st_ms, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clocks.summary(),
             "decode": decode, "select_stats": stats,

@@ -201,15 +201,33 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       issue(tile + NST - 1);
       const uint32_t sK = sKVa + (tile % NST) * 2 * SM::kTile;
       const uint32_t sV = sK + SM::kTile;
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // All K fragments first, then S = Q K^T in four independent accumulator
+      // chains (even / odd K slices), then the V fragments, whose latency the
+      // softmax below hides.
+      uint32_t kf[D / 16][4], vf[D / 16][4];
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t b[4];
         const int r = warp * 16 + (lane & 7) + (lane >> 4) * 8, c = kk * 2 + ((lane >> 3) & 1);
-        ldsm_x4(sK + kv_off<D>(r, c), b);
-        mma16816(s[0], qa[kk], b[0], b[1]);
-        mma16816(s[1], qa[kk], b[2], b[3]);
+        ldsm_x4(sK + kv_off<D>(r, c), kf[kk]);
       }
+      float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float sb[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        float (&acc)[2][4] = (kk & 1) ? sb : sa;
+        mma16816(acc[0], qa[kk], kf[kk][0], kf[kk][1]);
+        mma16816(acc[1], qa[kk], kf[kk][2], kf[kk][3]);
+      }
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt) {
+        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = dt * 2 + (lane >> 4);
+        ldsm_x4_t(sV + kv_off<D>(r, c), vf[dt]);
+      }
+      float s[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = sa[nt][e] + sb[nt][e];
       // scale (log2 domain) and mask keys past the end of this item's list
       const int key0 = tile * kKeysPerTile + warp * 16;
 #pragma unroll
@@ -262,11 +280,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       pa[3] = pack_bf16(pr[1][2], pr[1][3]);
 #pragma unroll
       for (int dt = 0; dt < D / 16; ++dt) {
-        uint32_t b[4];
-        const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8, c = dt * 2 + (lane >> 4);
-        ldsm_x4_t(sV + kv_off<D>(r, c), b);
-        mma16816(o[2 * dt], pa, b[0], b[1]);
-        mma16816(o[2 * dt + 1], pa, b[2], b[3]);
+        mma16816(o[2 * dt], pa, vf[dt][0], vf[dt][1]);
+        mma16816(o[2 * dt + 1], pa, vf[dt][2], vf[dt][3]);
       }
     }
     cp_async_wait<0>();

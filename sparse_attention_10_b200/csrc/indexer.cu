@@ -104,6 +104,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "r"(taddr));
 }
 
+// tcgen05.wait::ld that also names the 16 registers of the load it completes,
+// so the compiler keeps every use of them after the wait.
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                 "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                 "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
   const float f = __uint_as_float(acc_bits);
   return (f > 0.0f ? acc_bits : 0u) >> 16;  // non-negative float bits are monotone
@@ -320,62 +331,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt = item_ktile(p, qt, j, nt);
         const uint32_t tbase =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kBN + half * 128;
-#pragma unroll 1
-        for (int c = 0; c < 128 / kChunk; ++c) {
-          uint32_t v[kChunk];
-          tmem_ld16(tbase + c * kChunk, v);
-          tmem_ld_wait();
-          const int64_t s0 = static_cast<int64_t>(kt) * kBN + half * 128 + c * kChunk;
-          if (p.mode == kModeFilter) {
-            uint32_t pass = 0;
+        // Chunk c+1's TMEM load is in flight while chunk c is processed.
+        auto process = [&](int c, uint32_t (&v)[kChunk]) {
+            const int64_t s0 = static_cast<int64_t>(kt) * kBN + half * 128 + c * kChunk;
+            if (p.mode == kModeFilter) {
+              uint32_t pass = 0;
 #pragma unroll
-            for (int q = 0; q < kChunk; ++q) pass |= (__uint_as_float(v[q]) >= tau ? 1u : 0u) << q;
-            const int64_t lim = t - s0;  // keys s0 .. t are causal
-            if (lim < kChunk - 1) pass &= lim < 0 ? 0u : ((2u << lim) - 1u);
-            if (!row_ok) pass = 0;
-            if (pass) {
-              float4* st4 = reinterpret_cast<float4*>(my_stage);
+              for (int q = 0; q < kChunk; ++q) pass |= (__uint_as_float(v[q]) >= tau ? 1u : 0u) << q;
+              const int64_t lim = t - s0;  // keys s0 .. t are causal
+              if (lim < kChunk - 1) pass &= lim < 0 ? 0u : ((2u << lim) - 1u);
+              if (!row_ok) pass = 0;
+              if (pass) {
+                float4* st4 = reinterpret_cast<float4*>(my_stage);
 #pragma unroll
-              for (int q = 0; q < kChunk / 4; ++q)
-                st4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                     __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-              while (pass) {
-                const int q = __ffs(pass) - 1;
-                pass &= pass - 1;
-                float sc = __fmul_rn(my_stage[q], p.scale);
-                sc = sc > 0.0f ? sc : 0.0f;
-                const uint32_t s = static_cast<uint32_t>(s0 + q);
-                if (count < p.cap)
-                  my_cand[count] =
-                      (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xFFFFFFFFu - s);
-                ++count;
+                for (int q = 0; q < kChunk / 4; ++q)
+                  st4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                       __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+                while (pass) {
+                  const int q = __ffs(pass) - 1;
+                  pass &= pass - 1;
+                  float sc = __fmul_rn(my_stage[q], p.scale);
+                  sc = sc > 0.0f ? sc : 0.0f;
+                  const uint32_t s = static_cast<uint32_t>(s0 + q);
+                  if (count < p.cap)
+                    my_cand[count] =
+                        (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xFFFFFFFFu - s);
+                  ++count;
+                }
               }
-            }
-          } else if (p.mode == kModeSample) {
-            if (row_ok) {
-              uint32_t w[kChunk / 2];
+            } else if (p.mode == kModeSample) {
+              if (row_ok) {
+                uint32_t w[kChunk / 2];
 #pragma unroll
-              for (int q = 0; q < kChunk / 2; ++q)
-                w[q] = sample_key16(v[2 * q]) | (sample_key16(v[2 * q + 1]) << 16);
-              uint4* dst = reinterpret_cast<uint4*>(p.samp + t * p.samp_ld + j * kBN + half * 128 +
-                                                    c * kChunk);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-          } else {
-            if (row_ok) {
-              float* out = p.scores + t * p.Lk;
+                for (int q = 0; q < kChunk / 2; ++q)
+                  w[q] = sample_key16(v[2 * q]) | (sample_key16(v[2 * q + 1]) << 16);
+                uint4* dst = reinterpret_cast<uint4*>(p.samp + t * p.samp_ld + j * kBN + half * 128 +
+                                                      c * kChunk);
+                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              }
+            } else {
+              if (row_ok) {
+                float* out = p.scores + t * p.Lk;
 #pragma unroll
-              for (int q = 0; q < kChunk; ++q) {
-                const int64_t s = s0 + q;
-                if (s < p.Lk) {
-                  const float sc = __fmul_rn(__uint_as_float(v[q]), p.scale);
-                  out[s] = sc > 0.0f ? sc : 0.0f;
+                for (int q = 0; q < kChunk; ++q) {
+                  const int64_t s = s0 + q;
+                  if (s < p.Lk) {
+                    const float sc = __fmul_rn(__uint_as_float(v[q]), p.scale);
+                    out[s] = sc > 0.0f ? sc : 0.0f;
+                  }
                 }
               }
             }
-          }
+          };
+        uint32_t va[kChunk], vb[kChunk];
+        tmem_ld16(tbase, va);
+        tmem_ld_wait_regs(va);
+#pragma unroll
+        for (int c = 0; c < 128 / kChunk; c += 2) {
+          tmem_ld16(tbase + (c + 1) * kChunk, vb);
+          process(c, va);
           __syncwarp();
+          tmem_ld_wait_regs(vb);
+          if (c + 2 < 128 / kChunk) tmem_ld16(tbase + (c + 2) * kChunk, va);
+          process(c + 1, vb);
+          __syncwarp();
+          if (c + 2 < 128 / kChunk) tmem_ld_wait_regs(va);
         }
         tc_fence_before();
         __syncwarp();
