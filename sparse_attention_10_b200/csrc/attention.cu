@@ -163,20 +163,28 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     __syncthreads();
 
     const int ntiles = (n + kKeysPerTile - 1) / kKeysPerTile;
-    // Warp w copies key rows w, w+4, ...; its 32 lanes take the 16-byte pieces
-    // of one K row and one V row (coalesced 2D-byte rows).
+    // Eight lanes share a key: lane l8 copies 16-byte chunks l8, l8+8, ... of
+    // its K row and its V row (each group of eight lanes reads 128 contiguous
+    // bytes), with the row address computed once per key; a warp covers four
+    // keys per step.  Chunk c of row r lands at kv_off(r, c); with c = l8 + 8h
+    // that is the row's base + ((l8 ^ (r & 7)) << 4) + 128 h.
     auto issue = [&](int tile) {
       if (tile < ntiles) {
         const uint32_t st = sKVa + (tile % NST) * 2 * SM::kTile;
+        const int l8 = lane & 7, kq = lane >> 3;
 #pragma unroll
-        for (int u = 0; u < kKeysPerTile * 2 * PIECES / kAttnThreads; ++u) {
-          const int i = tid + u * kAttnThreads;
-          const int r = i / (2 * PIECES), rem = i % (2 * PIECES);
-          const int kv = rem / PIECES, c = rem % PIECES;
+        for (int it = 0; it < kKeysPerTile / 16; ++it) {
+          const int r = it * 16 + warp * 4 + kq;
           const int j = tile * kKeysPerTile + r;
           const int s = j < n ? sIds[j] : -1;
-          const __nv_bfloat16* src = (kv ? Vb : Kb) + static_cast<int64_t>(s < 0 ? 0 : s) * D + c * 8;
-          cp_async16(st + kv * SM::kTile + kv_off<D>(r, c), src, s < 0 ? 0u : 16u);
+          const uint32_t sz = s < 0 ? 0u : 16u;
+          const int64_t row = static_cast<int64_t>(s < 0 ? 0 : s) * D + l8 * 8;
+          const uint32_t dk = st + r * (2 * D) + ((l8 ^ (r & 7)) << 4);
+#pragma unroll
+          for (int h = 0; h < PIECES / 8; ++h) {
+            cp_async16(dk + h * 128, Kb + row + h * 64, sz);
+            cp_async16(dk + SM::kTile + h * 128, Vb + row + h * 64, sz);
+          }
         }
       }
       cp_async_commit();  // possibly empty: keeps one group per tile

@@ -13,8 +13,8 @@
 //   dense   write every score (check / small sizes only);
 //   sample  write 16-bit keys of the scores against a few evenly spaced key
 //           tiles, from which the per-row threshold is estimated;
-//   filter  keep (score, key) pairs whose raw accumulator reaches the row's
-//           threshold, appending them to the row's candidate list.
+//   filter  keep (raw accumulator, key) pairs whose accumulator reaches the
+//           row's threshold, appending them to the row's candidate list.
 // Causal: key tiles entirely above the diagonal are never issued; the
 // diagonal tile is masked per key in the epilogue.
 //
@@ -342,22 +342,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (lim < kChunk - 1) pass &= lim < 0 ? 0u : ((2u << lim) - 1u);
               if (!row_ok) pass = 0;
               if (pass) {
-                float4* st4 = reinterpret_cast<float4*>(my_stage);
+                // Each hit is stored as (raw accumulator bits, ~key); the select
+                // turns the accumulator into relu(fp32(acc) * scale).
+                const int hits = __popc(pass);
+                if (count + hits <= p.cap) {
+                  uint32_t* st = reinterpret_cast<uint32_t*>(my_stage);
+                  uint4* st4 = reinterpret_cast<uint4*>(my_stage);
 #pragma unroll
-                for (int q = 0; q < kChunk / 4; ++q)
-                  st4[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                       __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
-                while (pass) {
-                  const int q = __ffs(pass) - 1;
-                  pass &= pass - 1;
-                  float sc = __fmul_rn(my_stage[q], p.scale);
-                  sc = sc > 0.0f ? sc : 0.0f;
-                  const uint32_t s = static_cast<uint32_t>(s0 + q);
-                  if (count < p.cap)
-                    my_cand[count] =
-                        (static_cast<unsigned long long>(__float_as_uint(sc)) << 32) | (0xFFFFFFFFu - s);
-                  ++count;
+                  for (int q = 0; q < kChunk / 4; ++q)
+                    st4[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                  uint2* dst = reinterpret_cast<uint2*>(my_cand + count);
+                  const uint32_t nbase = 0xFFFFFFFFu - static_cast<uint32_t>(s0);
+                  while (pass) {
+                    const int q = __ffs(pass) - 1;
+                    pass &= pass - 1;
+                    *dst++ = make_uint2(nbase - q, st[q]);
+                  }
                 }
+                count += hits;
               }
             } else if (p.mode == kModeSample) {
               if (row_ok) {

@@ -2,20 +2,22 @@
 //
 // Token selection of the DeepSeek Sparse Attention page (kwkr.cn/news/60693,
 // section 3.3): query t keeps min(top_k, t+1) keys ranked by (score desc,
-// key index asc).  A candidate is one 64-bit key (score_bits << 32) |
-// (0xFFFFFFFF - s): scores are non-negative floats after ReLU, so their bits
-// order like the values, and the low word makes the lower key index win a
-// tie.  Larger key = better rank, all keys of a row are distinct.
+// key index asc).  The indexer stores each candidate as the 64-bit word
+// (raw accumulator bits << 32) | (0xFFFFFFFF - s), in two lists per row (one
+// per column half of its tile), each in ascending key order.
 //
-// select_kernel: one CTA per row; loads the row's two candidate lists (one
-// per indexer column half) into shared memory, finds the m-th largest key by
-// an 8-bit MSD radix select, compacts the m winners and sorts them (bitonic,
-// descending) into indices[t].  Rows whose lists overflowed, or hold fewer
-// than m keys, are queued for the fallback.
+// select_kernel: one CTA per row.  The two lists are merged into one
+// ascending-key run; the merge turns each accumulator into the score
+// relu(fp32(acc) * scale) (non-negative, so its bits order like the value).
+// Stable LSD radix passes over the score bytes that differ then order the
+// run by score, descending; equal scores keep ascending key order, so the
+// first min(top_k, t+1) entries are the answer.  Rows whose lists overflowed,
+// or hold fewer keys than needed, are queued for the fallback.
 //
 // fallback_kernel: recomputes every causal score of a queued row on CUDA
-// cores (sequential FP32 FMA, exact for integer-valued inputs), then runs the
-// same select over the whole row from a global scratch row.
+// cores (FP32, exact for integer-valued inputs), builds the 64-bit keys
+// (score_bits << 32) | (0xFFFFFFFF - s) -- larger key, better rank -- and
+// selects by MSD radix passes plus a bitonic sort of the winners.
 #include <cuda_fp8.h>
 
 #include <algorithm>
@@ -157,7 +159,7 @@ __device__ __forceinline__ uint32_t key_index(unsigned long long k) {
 // keys) into one ascending-index run, written as score words `sc` and key
 // indices `ix` (merge path: each thread finds its split by binary search).
 __device__ void merge_by_index(const unsigned long long* a, int na, const unsigned long long* b,
-                               int nb, uint32_t* sc, uint32_t* ix) {
+                               int nb, float scale, uint32_t* sc, uint32_t* ix) {
   const int n = na + nb;
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int p0 = min(n, static_cast<int>(threadIdx.x) * per), p1 = min(n, p0 + per);
@@ -174,7 +176,9 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
   for (int p = p0; p < p1; ++p) {
     const bool take_a = j >= nb || (i < na && key_index(a[i]) < key_index(b[j]));
     const unsigned long long k = take_a ? a[i++] : b[j++];
-    sc[p] = static_cast<uint32_t>(k >> 32);
+    // the filter stored the raw accumulator: score = relu(fp32(acc) * scale)
+    const float score = __fmul_rn(__uint_as_float(static_cast<uint32_t>(k >> 32)), scale);
+    sc[p] = score > 0.0f ? __float_as_uint(score) : 0u;
     ix[p] = key_index(k);
   }
 }
@@ -182,6 +186,7 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
 struct SelParams {
   int64_t L;
   int top_k, cap;
+  float scale;
   const unsigned long long* cand;
   const int* cand_n;
   const float* tau;
@@ -234,7 +239,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    merge_by_index(raw, n0, raw + n0, n1, sc0, ix);
+    merge_by_index(raw, n0, raw + n0, n1, p.scale, sc0, ix);
     __syncthreads();
     uint32_t o = 0u, a = 0xFFFFFFFFu, pos = 0u;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -416,7 +421,7 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
   if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
-  SelParams p{a.L, a.top_k, a.cap, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
+  SelParams p{a.L, a.top_k, a.cap, a.scale, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
   const size_t smem = static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
