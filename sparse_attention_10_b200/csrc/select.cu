@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
   uint32_t* cnt = ix + kSortCap;                                         // [warps][256] / bitmap
   uint32_t* base = cnt + kSortWarps * 256;                               // [256]
   uint32_t* misc = base + 256;                                           // [8]
+  // (positions of the merged run fit 16 bits: n <= kSortCap < 65536)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
@@ -225,9 +226,10 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     if (threadIdx.x == 0) {
       atomicAdd(&p.counters[2], n);
-      misc[0] = 0u;           // OR of score words
-      misc[1] = 0xFFFFFFFFu;  // AND of score words
+      misc[0] = 0u;           // OR of (score word - row minimum)
+      misc[1] = 0xFFFFFFFFu;  // AND of the same
       misc[2] = 0u;           // positive scores
+      misc[3] = 0xFFFFFFFFu;  // row minimum score word
     }
     const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
     const unsigned long long* c1 = c0 + p.cap;
@@ -241,20 +243,34 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     __syncthreads();
     merge_by_index(raw, n0, raw + n0, n1, p.scale, sc0, ix);
     __syncthreads();
-    uint32_t o = 0u, a = 0xFFFFFFFFu, pos = 0u;
+    // Score words of non-negative floats order like the values; subtracting
+    // the row minimum keeps the order and leaves fewer bytes to sort.
+    uint32_t lo = 0xFFFFFFFFu, pos = 0u;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t hi = sc0[i];
-      o |= hi;
-      a &= hi;
-      pos += hi != 0u;
+      const uint32_t w = sc0[i];
+      lo = min(lo, w);
+      pos += w != 0u;
+    }
+    lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+    pos = __reduce_add_sync(0xFFFFFFFFu, pos);
+    if (lane == 0) {
+      atomicMin(&misc[3], lo);
+      atomicAdd(&misc[2], pos);
+    }
+    __syncthreads();
+    const uint32_t row_min = misc[3];
+    uint32_t o = 0u, a = 0xFFFFFFFFu;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t w = sc0[i] - row_min;
+      sc0[i] = w;
+      o |= w;
+      a &= w;
     }
     o = __reduce_or_sync(0xFFFFFFFFu, o);
     a = __reduce_and_sync(0xFFFFFFFFu, a);
-    pos = __reduce_add_sync(0xFFFFFFFFu, pos);
     if (lane == 0) {
       atomicOr(&misc[0], o);
       atomicAnd(&misc[1], a);
-      atomicAdd(&misc[2], pos);
     }
     __syncthreads();
     const uint32_t vary = misc[0] ^ misc[1];
