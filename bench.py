@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample time")
     ap.add_argument("--workload", default=PREFILL,
-                    choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k"],
+                    choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k", "prefill_32k_bf16"],
                     help="prefill workload of a step (smaller ones for profiling)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="decode only the first B sequences of the batch (profiling)")

@@ -170,6 +170,8 @@ WORKLOADS = {
     "prefill_128k": Workload("prefill_128k", 4, "prefill", 131072, 160, "bf16", 16, 128, 2048),
     "decode_64x128k": Workload("decode_64x128k", 5, "decode", 0, 128, "fp8", 16, 128, 2048,
                                B=64, len_lo=65536, len_hi=131072),
+    # the 128K per-row settings at 32K length: a capture-sized stand-in for profiling
+    "prefill_32k_bf16": Workload("prefill_32k_bf16", 6, "prefill", 32768, 160, "bf16", 16, 128, 2048),
 }
 
 # tensor ids inside a workload's streams
