@@ -65,12 +65,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -242,25 +236,22 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[nt][e] = sa[nt][e] + sb[nt][e];
-      // Keys past the end of this item's list (only in a partial last tile).
+      // scale (log2 domain) and mask keys past the end of this item's list
       const int key0 = tile * kKeysPerTile + warp * 16;
-      if (key0 + 16 > n) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (key0 + nt * 8 + tig * 2 + (e & 1) >= n) s[nt][e] = -INFINITY;
-      }
-      // Row maxima of the raw logits (the scale is positive), then the
-      // running maxima m0/m1 in the scaled log2 domain: p = 2^(s*scale - m).
-      float mx0 = max3f(s[0][0], s[0][1], fmaxf(s[1][0], s[1][1]));
-      float mx1 = max3f(s[0][2], s[0][3], fmaxf(s[1][2], s[1][3]));
+        for (int e = 0; e < 4; ++e) {
+          const int j = key0 + nt * 8 + tig * 2 + (e & 1);
+          s[nt][e] = j < n ? s[nt][e] * p.scale_log2 : -INFINITY;
+        }
+      float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 1));
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xFFFFFFFFu, mx0, 2));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 1));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xFFFFFFFFu, mx1, 2));
-      const float sl = p.scale_log2;
-      const float n0 = fmaxf(m0, mx0 * sl), n1 = fmaxf(m1, mx1 * sl);
+      const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
       const float r0 = n0 == -INFINITY ? 0.0f : n0, r1 = n1 == -INFINITY ? 0.0f : n1;
       const bool same = n0 == m0 && n1 == m1;
       const float c0 = fast_exp2(m0 - r0), c1 = fast_exp2(m1 - r1);
@@ -269,10 +260,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       float pr[2][4];
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
-        pr[nt][0] = fast_exp2(fmaf(s[nt][0], sl, -r0));
-        pr[nt][1] = fast_exp2(fmaf(s[nt][1], sl, -r0));
-        pr[nt][2] = fast_exp2(fmaf(s[nt][2], sl, -r1));
-        pr[nt][3] = fast_exp2(fmaf(s[nt][3], sl, -r1));
+        pr[nt][0] = fast_exp2(s[nt][0] - r0);
+        pr[nt][1] = fast_exp2(s[nt][1] - r0);
+        pr[nt][2] = fast_exp2(s[nt][2] - r1);
+        pr[nt][3] = fast_exp2(s[nt][3] - r1);
       }
       const float ps0 = pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1];
       const float ps1 = pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3];

@@ -195,26 +195,21 @@ struct SelParams {
   int* counters;
 };
 
-// Bucket select of one row.  Keys (score_bits << 32) | ~index order every
-// candidate exactly as the output must (score desc, index asc), so no stable
-// pass is needed: keys go to 2048 buckets by the top bits of (max - score)
-// (bucket order = strictly descending score), each bucket that reaches into
-// the first m positions is sorted by its full key (insertion sort up to 32
-// keys, block-wide rank counting for larger, tie-heavy buckets), and the
-// first m keys are the answer.
-constexpr int kBuckets = 2048;
-constexpr int kSmallBucket = 32;
-
 __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long sel_smem[];
-  unsigned long long* raw = sel_smem;                               // [kSortCap] input, then scratch
-  unsigned long long* srt = raw + kSortCap;                         // [kSortCap] bucketed keys
-  uint32_t* hist = reinterpret_cast<uint32_t*>(srt + kSortCap);     // [kBuckets] sizes / bitmap
-  uint32_t* cur = hist + kBuckets;                                  // [kBuckets] offsets
-  uint32_t* wtot = cur + kBuckets;                                  // [kSortWarps]
-  uint32_t* misc = wtot + kSortWarps;                               // [16]
+  // raw: the row's two candidate lists (64-bit keys); after the merge the same
+  // bytes hold the second score buffer and both position buffers.
+  unsigned long long* raw = sel_smem;                                    // [kSortCap]
+  uint32_t* sc1 = reinterpret_cast<uint32_t*>(raw);                      // [kSortCap]
+  uint16_t* ps0 = reinterpret_cast<uint16_t*>(sc1 + kSortCap);           // [kSortCap]
+  uint16_t* ps1 = ps0 + kSortCap;                                        // [kSortCap]
+  uint32_t* sc0 = reinterpret_cast<uint32_t*>(raw + kSortCap);           // [kSortCap]
+  uint32_t* ix = sc0 + kSortCap;                                         // [kSortCap]
+  uint32_t* cnt = ix + kSortCap;                                         // [warps][256] / bitmap
+  uint32_t* base = cnt + kSortWarps * 256;                               // [256]
+  uint32_t* misc = base + 256;                                           // [8]
+  // (positions of the merged run fit 16 bits: n <= kSortCap < 65536)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
     const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
@@ -231,162 +226,73 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     if (threadIdx.x == 0) {
       atomicAdd(&p.counters[2], n);
-      misc[0] = 0xFFFFFFFFu;  // min score word
-      misc[1] = 0u;           // max score word
+      misc[0] = 0u;           // OR of (score word - row minimum)
+      misc[1] = 0xFFFFFFFFu;  // AND of the same
       misc[2] = 0u;           // positive scores
-      misc[3] = 0u;           // big buckets
+      misc[3] = 0xFFFFFFFFu;  // row minimum score word
     }
     const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
     const unsigned long long* c1 = c0 + p.cap;
+    // Both lists in flight at once (8-byte asynchronous copies), one wait.
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
       const unsigned long long* src = i < n0 ? c0 + i : c1 + (i - n0);
       asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(raw + i)), "l"(src)
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) hist[i] = 0u;
     __syncthreads();
-    // accumulator -> score relu(fp32(acc) * scale); key = (score_bits << 32) | ~index
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u, pos = 0u;
+    merge_by_index(raw, n0, raw + n0, n1, p.scale, sc0, ix);
+    __syncthreads();
+    // Score words of non-negative floats order like the values; subtracting
+    // the row minimum keeps the order and leaves fewer bytes to sort.
+    uint32_t lo = 0xFFFFFFFFu, pos = 0u;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const unsigned long long k = raw[i];
-      const float sc = __fmul_rn(__uint_as_float(static_cast<uint32_t>(k >> 32)), p.scale);
-      const uint32_t w = sc > 0.0f ? __float_as_uint(sc) : 0u;
-      raw[i] = (static_cast<unsigned long long>(w) << 32) | (k & 0xFFFFFFFFull);
+      const uint32_t w = sc0[i];
       lo = min(lo, w);
-      hi = max(hi, w);
       pos += w != 0u;
     }
     lo = __reduce_min_sync(0xFFFFFFFFu, lo);
-    hi = __reduce_max_sync(0xFFFFFFFFu, hi);
     pos = __reduce_add_sync(0xFFFFFFFFu, pos);
     if (lane == 0) {
-      atomicMin(&misc[0], lo);
-      atomicMax(&misc[1], hi);
+      atomicMin(&misc[3], lo);
       atomicAdd(&misc[2], pos);
     }
     __syncthreads();
-    const uint32_t wmax = misc[1];
-    const uint32_t range = wmax - misc[0];
-    const int shift = max(0, 32 - __clz(range) - 11);   // (range >> shift) < kBuckets
+    const uint32_t row_min = misc[3];
+    uint32_t o = 0u, a = 0xFFFFFFFFu;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t w = sc0[i] - row_min;
+      sc0[i] = w;
+      o |= w;
+      a &= w;
+    }
+    o = __reduce_or_sync(0xFFFFFFFFu, o);
+    a = __reduce_and_sync(0xFFFFFFFFu, a);
+    if (lane == 0) {
+      atomicOr(&misc[0], o);
+      atomicAnd(&misc[1], a);
+    }
+    __syncthreads();
+    const uint32_t vary = misc[0] ^ misc[1];
     const int npos = static_cast<int>(misc[2]);
-    const int iters = (n + blockDim.x - 1) / blockDim.x;
-    // bucket sizes (lanes with equal buckets add once)
-    for (int it = 0; it < iters; ++it) {
-      const int i = it * blockDim.x + threadIdx.x;
-      const uint32_t bk = i < n ? (wmax - static_cast<uint32_t>(raw[i] >> 32)) >> shift : 0xFFFFFFFFu;
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bk);
-      if (i < n && lane == __ffs(peers) - 1) atomicAdd(&hist[bk], __popc(peers));
-    }
-    __syncthreads();
-    {  // exclusive scan of the bucket sizes into cur (4 buckets per thread)
-      uint32_t v[4], sum = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        v[q] = hist[threadIdx.x * 4 + q];
-        sum += v[q];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      if (lane == 31) wtot[warp] = incl;
-      __syncthreads();
-      if (warp == 0) {
-        const uint32_t x = lane < kSortWarps ? wtot[lane] : 0u;
-        uint32_t wi = x;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
-          if (lane >= o) wi += y;
-        }
-        if (lane < kSortWarps) wtot[lane] = wi - x;
-      }
-      __syncthreads();
-      uint32_t ex = wtot[warp] + incl - sum;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        cur[threadIdx.x * 4 + q] = ex;
-        ex += v[q];
-      }
-    }
-    __syncthreads();
-    // scatter into buckets (order inside a bucket is arbitrary, fixed below)
-    for (int it = 0; it < iters; ++it) {
-      const int i = it * blockDim.x + threadIdx.x;
-      const unsigned long long k = i < n ? raw[i] : 0ull;
-      const uint32_t bk = i < n ? (wmax - static_cast<uint32_t>(k >> 32)) >> shift : 0xFFFFFFFFu;
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bk);
-      const int leader = __ffs(peers) - 1;
-      uint32_t b0 = 0;
-      if (i < n && lane == leader) b0 = atomicAdd(&cur[bk], __popc(peers));
-      b0 = __shfl_sync(0xFFFFFFFFu, b0, leader);
-      if (i < n) srt[b0 + __popc(peers & lt)] = k;
-    }
-    __syncthreads();
-    // sort the buckets that reach into the first m positions (cur = bucket end)
-    for (int bk = threadIdx.x; bk < kBuckets; bk += blockDim.x) {
-      const int size = static_cast<int>(hist[bk]);
-      const int st = static_cast<int>(cur[bk]) - size;
-      if (size < 2 || st >= m) continue;
-      if (size <= kSmallBucket) {
-        for (int i = st + 1; i < st + size; ++i) {
-          const unsigned long long k = srt[i];
-          int j = i - 1;
-          while (j >= st && srt[j] < k) {
-            srt[j + 1] = srt[j];
-            --j;
-          }
-          srt[j + 1] = k;
-        }
-      } else {
-        const uint32_t slot = atomicAdd(&misc[3], 1u);
-        if (slot < 8) misc[8 + slot] = static_cast<uint32_t>(bk);
-      }
-    }
-    __syncthreads();
-    const int nbig = static_cast<int>(misc[3]);
-    // Large buckets (many equal scores): rank of each key = keys above it.
-    // Up to eight are listed in misc[8..15]; with more, walk all buckets.
-    auto rank_sort = [&](int bk) {
-      const int size = static_cast<int>(hist[bk]);
-      const int st = static_cast<int>(cur[bk]) - size;
-      for (int i = threadIdx.x; i < size; i += blockDim.x) {
-        const unsigned long long k = srt[st + i];
-        int rank = 0;
-        for (int j = 0; j < size; ++j) rank += srt[st + j] > k;
-        raw[rank] = k;
-      }
-      __syncthreads();
-      for (int i = threadIdx.x; i < size; i += blockDim.x) srt[st + i] = raw[i];
-      __syncthreads();
-    };
-    if (nbig <= 8) {
-      for (int b = 0; b < nbig; ++b) rank_sort(static_cast<int>(misc[8 + b]));
-    } else {
-      for (int bk = 0; bk < kBuckets; ++bk) {
-        const int size = static_cast<int>(hist[bk]);
-        if (size > kSmallBucket && static_cast<int>(cur[bk]) - size < m) rank_sort(bk);
-      }
-    }
+    uint32_t* ks = sc0;
+    uint16_t* ps = nullptr;
+    stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary, cnt, base);
     int32_t* out = p.indices + t * p.top_k;
     if (!zero_mode || npos >= m) {
       for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
-        out[i] = i < m ? static_cast<int32_t>(key_index(srt[i])) : -1;
+        out[i] = i < m ? static_cast<int32_t>(ix[ps ? ps[i] : i]) : -1;
     } else {
       // Every positive score is a candidate; the rest of the row ranks the
       // zero scores by ascending key index.  Within keys [0, R) there are at
       // least m - npos zeros.
       const int R = static_cast<int>(min64(t + 1, static_cast<int64_t>(m) + npos));
       const int words = (R + 31) / 32;
-      uint32_t* bm = hist;
-      uint32_t* sc = cur;
+      uint32_t* bm = cnt;
       for (int wd = threadIdx.x; wd < words; wd += blockDim.x) bm[wd] = 0u;
       __syncthreads();
       for (int i = threadIdx.x; i < npos; i += blockDim.x) {
-        const uint32_t sidx = key_index(srt[i]);
+        const uint32_t sidx = ix[ps ? ps[i] : i];
         if (sidx < static_cast<uint32_t>(R)) atomicOr(&bm[sidx >> 5], 1u << (sidx & 31));
         out[i] = static_cast<int32_t>(sidx);
       }
@@ -404,15 +310,15 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
           const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
           if (lane >= off) incl += y;
         }
-        if (lane == 31) sc[warp] = incl;
+        if (lane == 31) base[warp] = incl;
         __syncwarp();
-        sc[8 + threadIdx.x] = incl - z;  // exclusive within the warp
+        base[8 + threadIdx.x] = incl - z;  // exclusive within the warp
       }
       __syncthreads();
       if (threadIdx.x < words) {
         const int wd = threadIdx.x;
-        uint32_t rank = sc[8 + wd];
-        for (int w2 = 0; w2 < warp; ++w2) rank += sc[w2];
+        uint32_t rank = base[8 + wd];
+        for (int w2 = 0; w2 < warp; ++w2) rank += base[w2];
         const uint32_t valid = (wd * 32 + 32 <= R) ? 0xFFFFFFFFu : ((1u << (R - wd * 32)) - 1u);
         uint32_t zeros = ~bm[wd] & valid;
         while (zeros) {
@@ -532,7 +438,7 @@ dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
   if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
   SelParams p{a.L, a.top_k, a.cap, a.scale, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
-  const size_t smem = static_cast<size_t>(kSortCap) * 16 + (2 * kBuckets + kSortWarps + 16) * 4;
+  const size_t smem = static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return DSA_ERR_CUDA;
