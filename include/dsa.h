@@ -183,6 +183,36 @@ dsa_status dsa_stage_times(double* ms, int64_t* launches, int n);
  */
 dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
+/*
+ * dsa_decode_static — dsa_decode for callers that cannot allocate device
+ * memory: a plugin whose host application owns every device allocation, or
+ * a serving loop that must not call cudaMalloc (it can synchronise the device
+ * and stall other streams) once it is running.  The pages describe no such
+ * entry point; it has no counterpart there.
+ *
+ * Arguments, outputs and errors are those of dsa_decode without the
+ * workspace: the scratch comes from one block of device memory built into
+ * the library (DSA_DECODE_STATIC_SCRATCH_BYTES = 18 MiB per device, held by
+ * every device that loads the library until the process exits).  That is
+ * enough for B <= 64 sequences holding up to 2^20 cached rows in total, with
+ * H <= 16, D <= 128, top_k <= 2048; sizes whose workspace
+ * (dsa_decode_workspace_size) exceeds it return DSA_ERR_WORKSPACE and enqueue
+ * nothing.  The caller still owns and passes every input and output.
+ *
+ * The first call on a device looks up that device's address of the block
+ * (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.  Every call on a device uses the same block and
+ * leaves its contents behind (each call clears what it needs zeroed), so
+ * calls whose work overlaps on the GPU — on different streams, or from
+ * different threads — race and corrupt each other: serialise them.
+ */
+#define DSA_DECODE_STATIC_SCRATCH_BYTES (18u << 20)
+dsa_status dsa_decode_static(const void* k_idx, const void* K, const void* V,
+                             const int64_t* seq_start, int B, int64_t total_rows, int64_t max_len,
+                             int idx_dtype, int d_idx, int D, const void* q_idx, const void* Q, int H,
+                             int top_k, float idx_scale, float attn_scale, void* O,
+                             int32_t* indices, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,7 +18,7 @@ __all__ = [
     "DsaError", "load", "dsa_version", "dsa_status_string", "dsa_indexer_scores",
     "dsa_prefill_workspace_size", "dsa_prefill", "dsa_decode_workspace_size", "dsa_decode",
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "IDX_FP8_E4M3", "IDX_BF16",
-    "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES",
+    "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -56,6 +56,7 @@ def load() -> ctypes.CDLL:
         "dsa_sync_status": ([P], I),
         "dsa_last_stats": ([P, ctypes.POINTER(ctypes.c_int64), P], I),
         "dsa_debug_wait_timeout": ([ctypes.c_uint64, P], I),
+        "dsa_decode_static": ([P, P, P, P, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P], I),
         "dsa_stage_timing": ([I], I),
         "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
     }
@@ -183,6 +184,28 @@ def dsa_decode(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_start:
                         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                         _stream(stream))
     _check(st, "dsa_decode")
+    return O, indices
+
+
+def dsa_decode_static(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_start: torch.Tensor,
+                      q_idx: torch.Tensor, Q: torch.Tensor, top_k: int, max_len: int,
+                      O: torch.Tensor, indices: Optional[torch.Tensor] = None,
+                      idx_scale: Optional[float] = None, attn_scale: Optional[float] = None,
+                      stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """dsa_decode with the library's built-in scratch: for callers that must not allocate.
+
+    O (and indices, if wanted) are passed in by the caller; nothing is allocated here.
+    """
+    lib = load()
+    B, d = q_idx.shape
+    _, H, D = Q.shape
+    if seq_start.dtype != torch.int64:
+        raise ValueError("seq_start must be int64")
+    st = lib.dsa_decode_static(_dev(k_idx, "k_idx"), _dev(K, "K"), _dev(V, "V"), _dev(seq_start, "seq_start"),
+                               B, k_idx.shape[0], int(max_len), _idx_dtype(q_idx), d, D, _dev(q_idx, "q_idx"),
+                               _dev(Q, "Q"), H, top_k, _scale(idx_scale), _scale(attn_scale), _dev(O, "O"),
+                               _dev(indices, "indices") if indices is not None else None, _stream(stream))
+    _check(st, "dsa_decode_static")
     return O, indices
 
 

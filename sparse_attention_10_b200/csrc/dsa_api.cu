@@ -471,3 +471,48 @@ dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ---- decode without allocation --------------------------------------------------------
+//
+// Scratch for dsa_decode_static: one block per device, in the library's own
+// device memory, so callers that may not allocate need no workspace.  Host
+// code cannot use the symbol's name as a device address; each device's
+// address is looked up once with cudaGetSymbolAddress while that device is
+// current.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_decode_static_scratch[DSA_DECODE_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_scratch[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" dsa_status dsa_decode_static(const void* k_idx, const void* K, const void* V,
+                                        const int64_t* seq_start, int B, int64_t total_rows,
+                                        int64_t max_len, int idx_dtype, int d_idx, int D,
+                                        const void* q_idx, const void* Q, int H, int top_k,
+                                        float idx_scale, float attn_scale, void* O,
+                                        int32_t* indices, void* stream) {
+  const size_t need = dsa_decode_workspace_size(B, total_rows, d_idx, idx_dtype, H, D, top_k);
+  if (need == 0) return DSA_ERR_INVALID_ARG;
+  if (need > DSA_DECODE_STATIC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> g(g_static_mu);
+    if (!g_static_scratch[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_decode_static_scratch) != cudaSuccess || !ptr)
+        return DSA_ERR_CUDA;
+      g_static_scratch[dev] = ptr;
+    }
+    scratch = g_static_scratch[dev];
+  }
+  return dsa_decode(k_idx, K, V, seq_start, B, total_rows, max_len, idx_dtype, d_idx, D, q_idx, Q,
+                    H, top_k, idx_scale, attn_scale, O, indices, scratch,
+                    DSA_DECODE_STATIC_SCRATCH_BYTES, stream);
+}
