@@ -189,6 +189,24 @@ __device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor for a K-major operand stored in swizzled
+// atoms of 8 rows: kind 0 = 128-byte rows (128-byte swizzle), 1 = 64-byte rows
+// (64-byte swizzle), 2 = 32-byte rows (32-byte swizzle).  The start address
+// may point 32 * k bytes into a row (the k-th 32-byte K step of the atom):
+// the swizzle is applied to the computed addresses, so the tile base must be
+// aligned to the atom (8 rows x row bytes).
+__device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, int kind) {
+  const uint32_t row_bytes = 128u >> kind;
+  const uint64_t layout = kind == 0 ? 2 : (kind == 1 ? 4 : 6);
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);          // start address
+  d |= static_cast<uint64_t>(1) << 16;                         // LBO (unused: K step fits a row)
+  d |= static_cast<uint64_t>((8 * row_bytes) >> 4) << 32;      // SBO: 8 rows
+  d |= static_cast<uint64_t>(1) << 46;                         // descriptor version (sm_100)
+  d |= layout << 61;                                           // swizzle mode
+  return d;
+}
+
 // Instruction descriptor: dense, FP32 accumulate, both operands K-major.
 // fmt 0 = E4M3 (kind::f8f6f4) or 1 = BF16 (kind::f16) for A and B.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t M, uint32_t N) {

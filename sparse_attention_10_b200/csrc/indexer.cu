@@ -44,10 +44,31 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTileA = kBM * 32;   // bytes of one 32-byte K slice of the A tile
 constexpr uint32_t kTileB = kBN * 32;   // bytes of one 32-byte K slice of a B tile
 
+// A row of d_bytes is split into column slices of 128 bytes (128-byte
+// swizzle), then at most one of 64 bytes (64-byte swizzle) and one of 32
+// bytes (32-byte swizzle); each slice is one TMA box per tile and gives
+// width/32 MMA K-steps.
+constexpr int kMaxSlices = 5;
+struct Slices {
+  int n;
+  int width[kMaxSlices];    // bytes: 128, 64 or 32
+  int col[kMaxSlices];      // byte offset of the slice in a row
+  int a_off[kMaxSlices];    // shared-memory offset of the slice in the A tile (128 rows)
+  int b_off[kMaxSlices];    // ... in a B stage (256 rows)
+  int kind[kMaxSlices];     // 0: 128-byte, 1: 64-byte, 2: 32-byte swizzle
+};
+
+struct Maps {                // tensor maps per swizzle kind
+  CUtensorMap q[3];          // query index rows, 128-row boxes
+  CUtensorMap k[3];          // key index rows, 256-row boxes
+  CUtensorMap k8[3];         // key index rows, 8-row boxes (sampled mini-tiles)
+};
+
 struct Params {
   const void* k_idx;
   int64_t Lq, Lk;
   int nkb, stages;
+  Slices sl;
   uint32_t off_b, off_stage, off_bar;
   float scale;
   int mode;
@@ -136,8 +157,7 @@ __device__ __forceinline__ int mini_tile_row(int64_t qt, int i, int nt) {
 
 template <int ESIZE>
 __global__ void __launch_bounds__(kThreads, 1)
-    indexer_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmK8, const Params p) {
+    indexer_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -172,8 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmK);
+    for (int i = 0; i < p.sl.n; ++i) {
+      tma_prefetch_desc(&maps.q[p.sl.kind[i]]);
+      tma_prefetch_desc(&maps.k[p.sl.kind[i]]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 2 * kBN);
@@ -202,9 +224,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(bar(A_EMPTY), (item_it & 1) ^ 1, p.limit_ns, abort_flag);
           if (ok) {
             mbar_arrive_expect_tx(bar(A_FULL), p.nkb * kTileA);
-            for (int b = 0; b < p.nkb; ++b)
-              tma_load_2d(sA + b * kTileA, &tmQ, b * (32 / ESIZE), static_cast<int>(qt * kBM),
-                          bar(A_FULL));
+            for (int i = 0; i < p.sl.n; ++i)
+              tma_load_2d(sA + p.sl.a_off[i], &maps.q[p.sl.kind[i]], p.sl.col[i] / ESIZE,
+                          static_cast<int>(qt * kBM), bar(A_FULL));
           }
         }
         if (gather) ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
@@ -219,17 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!gather) {
             mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
             const int kt = item_ktile(p, qt, j, nt);
-            for (int b = 0; b < p.nkb; ++b)
-              tma_load_2d(dst + b * kTileB, &tmK, b * (32 / ESIZE), kt * kBN, bar(FULL + s));
+            for (int i = 0; i < p.sl.n; ++i)
+              tma_load_2d(dst + p.sl.b_off[i], &maps.k[p.sl.kind[i]], p.sl.col[i] / ESIZE, kt * kBN,
+                          bar(FULL + s));
           } else {
             // 32 mini-tiles of 8 consecutive keys; each lane loads one mini-tile
             // (all 32-byte slices) into rows 8*lane .. 8*lane+7 of the stage.
             if (lane == 0) mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
             __syncwarp();
             const int y = mini_tile_row(qt, j * kMinisPerTile + lane, nt);
-            for (int b = 0; b < p.nkb; ++b)
-              tma_load_2d(dst + b * kTileB + lane * kMiniRows * 32, &tmK8, b * (32 / ESIZE), y,
-                          bar(FULL + s));
+            for (int i = 0; i < p.sl.n; ++i)
+              tma_load_2d(dst + p.sl.b_off[i] + lane * kMiniRows * p.sl.width[i], &maps.k8[p.sl.kind[i]],
+                          p.sl.col[i] / ESIZE, y, bar(FULL + s));
           }
           ++it;
         }
@@ -277,13 +300,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + buf * kBN;
           const uint32_t bstage = sB + s * stage_bytes;
-          for (int b = 0; b < p.nkb; ++b) {
-            const uint64_t ad = smem_desc_sw32(sA + b * kTileA);
-            const uint64_t bd = smem_desc_sw32(bstage + b * kTileB);
-            if (ESIZE == 1)
-              mma_f8(d_tmem, ad, bd, idesc, b > 0 ? 1u : 0u);
-            else
-              mma_bf16(d_tmem, ad, bd, idesc, b > 0 ? 1u : 0u);
+          uint32_t acc = 0;
+          for (int i = 0; i < p.sl.n; ++i) {
+            for (int k = 0; k < p.sl.width[i]; k += 32) {  // one MMA per 32 bytes of K
+              const uint64_t ad = smem_desc_kmajor(sA + p.sl.a_off[i] + k, p.sl.kind[i]);
+              const uint64_t bd = smem_desc_kmajor(bstage + p.sl.b_off[i] + k, p.sl.kind[i]);
+              if (ESIZE == 1)
+                mma_f8(d_tmem, ad, bd, idesc, acc);
+              else
+                mma_bf16(d_tmem, ad, bd, idesc, acc);
+              acc = 1;
+            }
           }
           mma_commit(bar(EMPTY + s));
           mma_commit(bar(ACC_FULL + buf));
@@ -531,19 +558,41 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major [rows, d] matrix, boxes of 32 bytes x box_rows, 32-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int esize, int d, int64_t rows, int box_rows) {
+// Row-major [rows, d] matrix, boxes of `width` bytes x box_rows, swizzle
+// matching the width (128, 64 or 32 bytes).
+bool make_map(CUtensorMap* m, const void* base, int esize, int d, int64_t rows, int box_rows,
+              int width) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * esize};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(32 / esize), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(width / esize), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = width == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : width == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = fn(m, esize == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
-                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+Slices make_slices(int d_bytes) {
+  Slices sl{};
+  int col = 0;
+  auto add = [&](int w, int kind) {
+    sl.width[sl.n] = w;
+    sl.col[sl.n] = col;
+    sl.a_off[sl.n] = col * kBM;
+    sl.b_off[sl.n] = col * kBN;
+    sl.kind[sl.n] = kind;
+    ++sl.n;
+    col += w;
+  };
+  while (d_bytes - col >= 128) add(128, 0);
+  if (d_bytes - col >= 64) add(64, 1);
+  if (d_bytes - col >= 32) add(32, 2);
+  return sl;
 }
 
 }  // namespace
@@ -580,22 +629,30 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   // At least 116 KB so two CTAs never share an SM (each holds all 512 TMEM columns).
   const size_t smem = std::max<size_t>(p.off_bar + kMiscBytes + 1024, 116 * 1024);
 
-  CUtensorMap tmQ, tmK, tmK8;
-  if (!make_map(&tmQ, a.q_idx, a.esize, a.d, a.Lq, kBM) ||
-      !make_map(&tmK, a.k_idx, a.esize, a.d, a.Lk, kBN) ||
-      !make_map(&tmK8, a.k_idx, a.esize, a.d, a.Lk, kMiniRows))
-    return DSA_ERR_CUDA;
+  p.sl = make_slices(d_bytes);
+  Maps maps{};
+  const int widths[3] = {128, 64, 32};
+  for (int kind = 0; kind < 3; ++kind) {
+    bool used = false;
+    for (int i = 0; i < p.sl.n; ++i) used |= p.sl.kind[i] == kind;
+    if (!used) continue;  // maps of unused kinds stay zero and are never read
+    const int w = widths[kind];
+    if (!make_map(&maps.q[kind], a.q_idx, a.esize, a.d, a.Lq, kBM, w) ||
+        !make_map(&maps.k[kind], a.k_idx, a.esize, a.d, a.Lk, kBN, w) ||
+        !make_map(&maps.k8[kind], a.k_idx, a.esize, a.d, a.Lk, kMiniRows, w))
+      return DSA_ERR_CUDA;
+  }
 
   const int grid = std::max(1, std::min(p.n_items, num_sms()));
   cudaError_t e;
   if (a.esize == 1) {
     e = cudaFuncSetAttribute(indexer_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-    if (e == cudaSuccess) indexer_kernel<1><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmK8, p);
+    if (e == cudaSuccess) indexer_kernel<1><<<grid, kThreads, smem, stream>>>(maps, p);
   } else {
     e = cudaFuncSetAttribute(indexer_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
-    if (e == cudaSuccess) indexer_kernel<2><<<grid, kThreads, smem, stream>>>(tmQ, tmK, tmK8, p);
+    if (e == cudaSuccess) indexer_kernel<2><<<grid, kThreads, smem, stream>>>(maps, p);
   }
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
