@@ -136,6 +136,33 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&v)[16]) {
                : "memory");
 }
 
+// tcgen05.wait::ld naming all 128 registers of a warp's strip (see above).
+__device__ __forceinline__ void tmem_ld_wait_all(uint32_t (&v)[8][16]) {
+#pragma unroll
+  for (int c = 0; c < 8; c += 2) {
+    asm volatile("" : "+r"(v[c][0]), "+r"(v[c][1]), "+r"(v[c][2]), "+r"(v[c][3]), "+r"(v[c][4]),
+                 "+r"(v[c][5]), "+r"(v[c][6]), "+r"(v[c][7]), "+r"(v[c][8]), "+r"(v[c][9]),
+                 "+r"(v[c][10]), "+r"(v[c][11]), "+r"(v[c][12]), "+r"(v[c][13]), "+r"(v[c][14]),
+                 "+r"(v[c][15]), "+r"(v[c + 1][0]), "+r"(v[c + 1][1]), "+r"(v[c + 1][2]),
+                 "+r"(v[c + 1][3]), "+r"(v[c + 1][4]), "+r"(v[c + 1][5]), "+r"(v[c + 1][6]),
+                 "+r"(v[c + 1][7]), "+r"(v[c + 1][8]), "+r"(v[c + 1][9]), "+r"(v[c + 1][10]),
+                 "+r"(v[c + 1][11]), "+r"(v[c + 1][12]), "+r"(v[c + 1][13]), "+r"(v[c + 1][14]),
+                 "+r"(v[c + 1][15]));
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int c = 0; c < 8; c += 2) {
+    asm volatile("" : "+r"(v[c][0]), "+r"(v[c][1]), "+r"(v[c][2]), "+r"(v[c][3]), "+r"(v[c][4]),
+                 "+r"(v[c][5]), "+r"(v[c][6]), "+r"(v[c][7]), "+r"(v[c][8]), "+r"(v[c][9]),
+                 "+r"(v[c][10]), "+r"(v[c][11]), "+r"(v[c][12]), "+r"(v[c][13]), "+r"(v[c][14]),
+                 "+r"(v[c][15]), "+r"(v[c + 1][0]), "+r"(v[c + 1][1]), "+r"(v[c + 1][2]),
+                 "+r"(v[c + 1][3]), "+r"(v[c + 1][4]), "+r"(v[c + 1][5]), "+r"(v[c + 1][6]),
+                 "+r"(v[c + 1][7]), "+r"(v[c + 1][8]), "+r"(v[c + 1][9]), "+r"(v[c + 1][10]),
+                 "+r"(v[c + 1][11]), "+r"(v[c + 1][12]), "+r"(v[c + 1][13]), "+r"(v[c + 1][14]),
+                 "+r"(v[c + 1][15]));
+  }
+}
+
 __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
   const float f = __uint_as_float(acc_bits);
   return (f > 0.0f ? acc_bits : 0u) >> 16;  // non-negative float bits are monotone
@@ -358,7 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt = item_ktile(p, qt, j, nt);
         const uint32_t tbase =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kBN + half * 128;
-        // Chunk c+1's TMEM load is in flight while chunk c is processed.
+        // The warp's whole 128-column strip: 8 loads in flight, one wait, then
+        // the accumulator goes back to the MMA warp before the values are used.
         auto process = [&](int c, uint32_t (&v)[kChunk]) {
             const int64_t s0 = static_cast<int64_t>(kt) * kBN + half * 128 + c * kChunk;
             if (p.mode == kModeFilter) {
@@ -413,23 +441,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           };
-        uint32_t va[kChunk], vb[kChunk];
-        tmem_ld16(tbase, va);
-        tmem_ld_wait_regs(va);
+        uint32_t vals[128 / kChunk][kChunk];
 #pragma unroll
-        for (int c = 0; c < 128 / kChunk; c += 2) {
-          tmem_ld16(tbase + (c + 1) * kChunk, vb);
-          process(c, va);
-          __syncwarp();
-          tmem_ld_wait_regs(vb);
-          if (c + 2 < 128 / kChunk) tmem_ld16(tbase + (c + 2) * kChunk, va);
-          process(c + 1, vb);
-          __syncwarp();
-          if (c + 2 < 128 / kChunk) tmem_ld_wait_regs(va);
-        }
+        for (int c = 0; c < 128 / kChunk; ++c) tmem_ld16(tbase + c * kChunk, vals[c]);
+        tmem_ld_wait_all(vals);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(ACC_EMPTY + buf));
+#pragma unroll
+        for (int c = 0; c < 128 / kChunk; ++c) {
+          process(c, vals[c]);
+          __syncwarp();
+        }
         ++acc_it;
       }
       if (!ok) break;
