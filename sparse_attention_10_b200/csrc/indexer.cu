@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float tau = INFINITY;
       if (p.mode == kModeFilter && row_ok) tau = p.tau[t];
       int count = 0;
+      uint32_t ring[6];  // up to three pending (key, accumulator) hits of this row
       unsigned long long* my_cand =
           p.mode == kModeFilter && row_ok ? p.cand + (2 * t + half) * static_cast<int64_t>(p.cap)
                                           : nullptr;
@@ -399,6 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (pass) {
                 // Each hit is stored as (raw accumulator bits, ~key); the select
                 // turns the accumulator into relu(fp32(acc) * scale).
+                // Hits wait in registers (ring of 3) and leave four at a time as
+                // two 16-byte stores at a 32-byte-aligned list position.
                 const int hits = __popc(pass);
                 if (count + hits <= p.cap) {
                   uint32_t* st = reinterpret_cast<uint32_t*>(my_stage);
@@ -406,15 +409,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                   for (int q = 0; q < kChunk / 4; ++q)
                     st4[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-                  uint2* dst = reinterpret_cast<uint2*>(my_cand + count);
                   const uint32_t nbase = 0xFFFFFFFFu - static_cast<uint32_t>(s0);
                   while (pass) {
                     const int q = __ffs(pass) - 1;
                     pass &= pass - 1;
-                    *dst++ = make_uint2(nbase - q, st[q]);
+                    const uint32_t key = nbase - q, acc = st[q];
+                    const int slot = count & 3;
+                    if (slot == 3) {
+                      uint4* dst = reinterpret_cast<uint4*>(my_cand + (count - 3));
+                      dst[0] = make_uint4(ring[0], ring[1], ring[2], ring[3]);
+                      dst[1] = make_uint4(ring[4], ring[5], key, acc);
+                    } else {
+                      if (slot == 0) { ring[0] = key; ring[1] = acc; }
+                      if (slot == 1) { ring[2] = key; ring[3] = acc; }
+                      if (slot == 2) { ring[4] = key; ring[5] = acc; }
+                    }
+                    ++count;
                   }
+                } else {
+                  count += hits;
                 }
-                count += hits;
               }
             } else if (p.mode == kModeSample) {
               if (row_ok) {
@@ -456,7 +470,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++acc_it;
       }
       if (!ok) break;
-      if (p.mode == kModeFilter && row_ok) p.cand_n[2 * t + half] = count;
+      if (p.mode == kModeFilter && row_ok) {
+        if (count <= p.cap) {  // the last (count & 3) hits are still in the ring
+          const int pend = count & 3;
+          uint2* dst = reinterpret_cast<uint2*>(my_cand + (count - pend));
+          if (pend > 0) dst[0] = make_uint2(ring[0], ring[1]);
+          if (pend > 1) dst[1] = make_uint2(ring[2], ring[3]);
+          if (pend > 2) dst[2] = make_uint2(ring[4], ring[5]);
+        }
+        p.cand_n[2 * t + half] = count;
+      }
     }
   }
 
