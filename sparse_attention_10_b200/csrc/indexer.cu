@@ -136,33 +136,6 @@ __device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&v)[16]) {
                : "memory");
 }
 
-// tcgen05.wait::ld naming all 128 registers of a warp's strip (see above).
-__device__ __forceinline__ void tmem_ld_wait_all(uint32_t (&v)[8][16]) {
-#pragma unroll
-  for (int c = 0; c < 8; c += 2) {
-    asm volatile("" : "+r"(v[c][0]), "+r"(v[c][1]), "+r"(v[c][2]), "+r"(v[c][3]), "+r"(v[c][4]),
-                 "+r"(v[c][5]), "+r"(v[c][6]), "+r"(v[c][7]), "+r"(v[c][8]), "+r"(v[c][9]),
-                 "+r"(v[c][10]), "+r"(v[c][11]), "+r"(v[c][12]), "+r"(v[c][13]), "+r"(v[c][14]),
-                 "+r"(v[c][15]), "+r"(v[c + 1][0]), "+r"(v[c + 1][1]), "+r"(v[c + 1][2]),
-                 "+r"(v[c + 1][3]), "+r"(v[c + 1][4]), "+r"(v[c + 1][5]), "+r"(v[c + 1][6]),
-                 "+r"(v[c + 1][7]), "+r"(v[c + 1][8]), "+r"(v[c + 1][9]), "+r"(v[c + 1][10]),
-                 "+r"(v[c + 1][11]), "+r"(v[c + 1][12]), "+r"(v[c + 1][13]), "+r"(v[c + 1][14]),
-                 "+r"(v[c + 1][15]));
-  }
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int c = 0; c < 8; c += 2) {
-    asm volatile("" : "+r"(v[c][0]), "+r"(v[c][1]), "+r"(v[c][2]), "+r"(v[c][3]), "+r"(v[c][4]),
-                 "+r"(v[c][5]), "+r"(v[c][6]), "+r"(v[c][7]), "+r"(v[c][8]), "+r"(v[c][9]),
-                 "+r"(v[c][10]), "+r"(v[c][11]), "+r"(v[c][12]), "+r"(v[c][13]), "+r"(v[c][14]),
-                 "+r"(v[c][15]), "+r"(v[c + 1][0]), "+r"(v[c + 1][1]), "+r"(v[c + 1][2]),
-                 "+r"(v[c + 1][3]), "+r"(v[c + 1][4]), "+r"(v[c + 1][5]), "+r"(v[c + 1][6]),
-                 "+r"(v[c + 1][7]), "+r"(v[c + 1][8]), "+r"(v[c + 1][9]), "+r"(v[c + 1][10]),
-                 "+r"(v[c + 1][11]), "+r"(v[c + 1][12]), "+r"(v[c + 1][13]), "+r"(v[c + 1][14]),
-                 "+r"(v[c + 1][15]));
-  }
-}
-
 __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
   const float f = __uint_as_float(acc_bits);
   return (f > 0.0f ? acc_bits : 0u) >> 16;  // non-negative float bits are monotone
@@ -372,7 +345,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       float tau = INFINITY;
       if (p.mode == kModeFilter && row_ok) tau = p.tau[t];
       int count = 0;
-      uint32_t ring[6];  // up to three pending (key, accumulator) hits of this row
       unsigned long long* my_cand =
           p.mode == kModeFilter && row_ok ? p.cand + (2 * t + half) * static_cast<int64_t>(p.cap)
                                           : nullptr;
@@ -386,8 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kt = item_ktile(p, qt, j, nt);
         const uint32_t tbase =
             tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kBN + half * 128;
-        // The warp's whole 128-column strip: 8 loads in flight, one wait, then
-        // the accumulator goes back to the MMA warp before the values are used.
+        // Chunk c+1's TMEM load is in flight while chunk c is processed.
         auto process = [&](int c, uint32_t (&v)[kChunk]) {
             const int64_t s0 = static_cast<int64_t>(kt) * kBN + half * 128 + c * kChunk;
             if (p.mode == kModeFilter) {
@@ -400,8 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (pass) {
                 // Each hit is stored as (raw accumulator bits, ~key); the select
                 // turns the accumulator into relu(fp32(acc) * scale).
-                // Hits wait in registers (ring of 3) and leave four at a time as
-                // two 16-byte stores at a 32-byte-aligned list position.
                 const int hits = __popc(pass);
                 if (count + hits <= p.cap) {
                   uint32_t* st = reinterpret_cast<uint32_t*>(my_stage);
@@ -409,26 +378,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                   for (int q = 0; q < kChunk / 4; ++q)
                     st4[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                  uint2* dst = reinterpret_cast<uint2*>(my_cand + count);
                   const uint32_t nbase = 0xFFFFFFFFu - static_cast<uint32_t>(s0);
                   while (pass) {
                     const int q = __ffs(pass) - 1;
                     pass &= pass - 1;
-                    const uint32_t key = nbase - q, acc = st[q];
-                    const int slot = count & 3;
-                    if (slot == 3) {
-                      uint4* dst = reinterpret_cast<uint4*>(my_cand + (count - 3));
-                      dst[0] = make_uint4(ring[0], ring[1], ring[2], ring[3]);
-                      dst[1] = make_uint4(ring[4], ring[5], key, acc);
-                    } else {
-                      if (slot == 0) { ring[0] = key; ring[1] = acc; }
-                      if (slot == 1) { ring[2] = key; ring[3] = acc; }
-                      if (slot == 2) { ring[4] = key; ring[5] = acc; }
-                    }
-                    ++count;
+                    *dst++ = make_uint2(nbase - q, st[q]);
                   }
-                } else {
-                  count += hits;
                 }
+                count += hits;
               }
             } else if (p.mode == kModeSample) {
               if (row_ok) {
@@ -455,31 +413,27 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           };
-        uint32_t vals[128 / kChunk][kChunk];
+        uint32_t va[kChunk], vb[kChunk];
+        tmem_ld16(tbase, va);
+        tmem_ld_wait_regs(va);
 #pragma unroll
-        for (int c = 0; c < 128 / kChunk; ++c) tmem_ld16(tbase + c * kChunk, vals[c]);
-        tmem_ld_wait_all(vals);
+        for (int c = 0; c < 128 / kChunk; c += 2) {
+          tmem_ld16(tbase + (c + 1) * kChunk, vb);
+          process(c, va);
+          __syncwarp();
+          tmem_ld_wait_regs(vb);
+          if (c + 2 < 128 / kChunk) tmem_ld16(tbase + (c + 2) * kChunk, va);
+          process(c + 1, vb);
+          __syncwarp();
+          if (c + 2 < 128 / kChunk) tmem_ld_wait_regs(va);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(ACC_EMPTY + buf));
-#pragma unroll
-        for (int c = 0; c < 128 / kChunk; ++c) {
-          process(c, vals[c]);
-          __syncwarp();
-        }
         ++acc_it;
       }
       if (!ok) break;
-      if (p.mode == kModeFilter && row_ok) {
-        if (count <= p.cap) {  // the last (count & 3) hits are still in the ring
-          const int pend = count & 3;
-          uint2* dst = reinterpret_cast<uint2*>(my_cand + (count - pend));
-          if (pend > 0) dst[0] = make_uint2(ring[0], ring[1]);
-          if (pend > 1) dst[1] = make_uint2(ring[2], ring[3]);
-          if (pend > 2) dst[2] = make_uint2(ring[4], ring[5]);
-        }
-        p.cand_n[2 * t + half] = count;
-      }
+      if (p.mode == kModeFilter && row_ok) p.cand_n[2 * t + half] = count;
     }
   }
 
