@@ -371,6 +371,15 @@ __global__ void __launch_bounds__(D) combine_kernel(const float* part, int nspli
   O[(q * H + h) * D + col] = __float2bfloat16_rn(den > 0.0f ? num / den : 0.0f);
 }
 
+// Split partials -> final output (nothing to do with one split).
+template <int D>
+dsa_status launch_combine(const AttnLaunch& a, cudaStream_t stream) {
+  if (a.nsplit == 1) return DSA_OK;
+  combine_kernel<D><<<static_cast<unsigned int>(a.nq * a.H), D, 0, stream>>>(a.part, a.nsplit, a.H,
+                                                                             a.O, a.invalid);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
 template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p{a.Q, a.K, a.V, a.idx, a.ld_idx, a.nq, a.H, a.scale_log2, a.top_k, a.seq_start,
@@ -388,17 +397,16 @@ dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   const int grid = static_cast<int>(std::min<int64_t>(items, std::max(1, per_sm) * num_sms()));
   attn_kernel<D><<<grid, kAttnThreads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  if (a.nsplit > 1) {
-    combine_kernel<D><<<static_cast<unsigned int>(a.nq * a.H), D, 0, stream>>>(a.part, a.nsplit,
-                                                                               a.H, a.O, a.invalid);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
-  }
-  return DSA_OK;
+  return launch_combine<D>(a, stream);
 }
 
 }  // namespace
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream) {
+  if (attention_tc_supported(a)) {
+    const dsa_status st = launch_attention_tc(a, stream);
+    return st != DSA_OK ? st : launch_combine<128>(a, stream);
+  }
   if (a.D == 64) return launch_d<64>(a, stream);
   if (a.D == 128) return launch_d<128>(a, stream);
   return DSA_ERR_UNSUPPORTED;

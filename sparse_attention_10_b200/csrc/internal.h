@@ -92,6 +92,11 @@ struct AttnLaunch {
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream);
 
+// tcgen05 attention (head dim 128, up to 16 heads); launch_attention routes
+// the shapes it supports there.
+bool attention_tc_supported(const AttnLaunch& a);
+dsa_status launch_attention_tc(const AttnLaunch& a, cudaStream_t stream);
+
 // ---- decode ------------------------------------------------------------------
 
 struct DecodeLaunch {
