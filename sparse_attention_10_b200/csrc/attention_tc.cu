@@ -124,15 +124,16 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
                "r"(src_bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
 }
-// Generic-proxy writes of this thread (stores, completed cp.async) become
-// visible to the tensor cores' (async proxy) reads that follow.
+// This thread's shared-memory stores become visible to the tensor cores'
+// (async proxy) reads that follow.
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -268,69 +269,91 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
     // Eight lanes per key row: lane l8 copies 16-byte chunks l8 (dims 0..63)
     // and l8 + 8 (dims 64..127); chunk c of row r goes to atom c / 8 at
     // r * 128 + ((c % 8) ^ (r % 8)) * 16.  A warp covers four rows per step.
+    // Key ids live in registers: for tile kt, lane L of gather warp pw holds
+    // the id (or -1) of key kt * 128 + (L / 4) * 16 + pw * 4 + L % 4 (the
+    // keys this warp copies) and hands it to the copying lanes by shuffle.
+    // The next item's ids are loaded while the current item is copied.  Each
+    // thread's copies of a tile are tracked by an asynchronous arrival on the
+    // tile's FULL barrier (cp.async.mbarrier.arrive.noinc, 128 expected), so
+    // the gather never waits for its own copies.
     const int pw = warp - 4, l8 = lane & 7, kq = lane >> 3;
     const int pt = pw * 32 + lane;
     uint32_t g = 0, ait = 0;
-    bool ok = true;
-    for (int64_t item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const Item it = make_item(p, item);
-      const int nt = (it.n + kKeys - 1) / kKeys;
-      if (nt == 0) continue;
-      if (!mbar_wait(bar(Q_EMPTY), (ait & 1) ^ 1, p.limit_ns, abort_flag)) {
-        ok = false;
-        break;
+    auto find = [&](int64_t& scan, Item& it, int& nt) -> bool {
+      for (; scan < n_items; scan += gridDim.x) {
+        it = make_item(p, scan);
+        nt = (it.n + kKeys - 1) / kKeys;
+        if (nt > 0) {
+          scan += gridDim.x;
+          return true;
+        }
       }
-      // Q rows (heads >= H zero), same 128-byte-swizzled K-major layout.
+      return false;
+    };
+    auto load_ids = [&](const Item& it, int nt, int32_t (&v)[kMaxTiles]) {
+#pragma unroll
+      for (int kt = 0; kt < kMaxTiles; ++kt) {
+        const int j = kt * kKeys + (lane >> 2) * 16 + pw * 4 + (lane & 3);
+        v[kt] = kt < nt && j < it.n ? __ldg(it.ids + j) : -1;
+      }
+    };
+    // one tile: K or V rows of keys kt * 128 .. +127 into the next stage
+    auto tile = [&](const __nv_bfloat16* src, int32_t my_id, bool with_q) -> bool {
+      const uint32_t stage = g % kNst;
+      if (!mbar_wait(bar(EMPTY + stage), ((g / kNst) & 1) ^ 1, p.limit_ns, abort_flag))
+        return false;
+      const uint32_t dst = sRing + stage * kTileBytes;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        const int r = s * 16 + pw * 4 + kq;
+        const int32_t id = __shfl_sync(0xFFFFFFFFu, my_id, s * 4 + kq);
+        const __nv_bfloat16* row = src + static_cast<int64_t>(id < 0 ? 0 : id) * kD + l8 * 8;
+        const uint32_t d = dst + r * 128 + ((l8 ^ (r & 7)) << 4);
+        cp_async16(d, row, id < 0 ? 0u : 16u);
+        cp_async16(d + kKeys * 128, row + 64, id < 0 ? 0u : 16u);
+      }
+      cp_async_arrive(bar(FULL + stage));
+      if (with_q) cp_async_arrive(bar(Q_FULL));
+      ++g;
+      return true;
+    };
+    int64_t scan = blockIdx.x;
+    Item cur{}, nxt{};
+    int cur_nt = 0, nxt_nt = 0;
+    int32_t ids[kMaxTiles], nids[kMaxTiles];
+    bool have = find(scan, cur, cur_nt);
+    if (have) load_ids(cur, cur_nt, ids);
+    bool ok = true;
+    while (have && ok) {
+      const bool have_nxt = find(scan, nxt, nxt_nt);
+      if (have_nxt) load_ids(nxt, nxt_nt, nids);
+#pragma unroll
+      for (int kt = 0; kt < kMaxTiles; ++kt)
+        ids[kt] = ids[kt] >= 0 && ids[kt] < cur.row_limit ? ids[kt] : -1;
+      if (!mbar_wait(bar(Q_EMPTY), (ait & 1) ^ 1, p.limit_ns, abort_flag)) break;
+      // Q rows (heads >= H zero), same 128-byte-swizzled K-major layout; they
+      // complete with the first K tile.
       for (int i = pt; i < kN * 16; i += 128) {
         const int h = i >> 4, c = i & 15;
         cp_async16(sQ + (c >> 3) * (kN * 128) + h * 128 + (((c & 7) ^ (h & 7)) << 4),
-                   p.Q + (it.q * p.H + min(h, p.H - 1)) * kD + c * 8, h < p.H ? 16u : 0u);
+                   p.Q + (cur.q * p.H + min(h, p.H - 1)) * kD + c * 8, h < p.H ? 16u : 0u);
       }
-      const __nv_bfloat16* Kb = p.K + it.row_base * kD;
-      const __nv_bfloat16* Vb = p.V + it.row_base * kD;
-      uint32_t prev_stage = 0;
-      for (int u = 0; u < 2 * nt; ++u) {
-        const int kt = u < nt ? u : u - nt;
-        const __nv_bfloat16* src = u < nt ? Kb : Vb;
-        int32_t id[8];
+      const __nv_bfloat16* Kb = p.K + cur.row_base * kD;
+      const __nv_bfloat16* Vb = p.V + cur.row_base * kD;
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int j = kt * kKeys + s * 16 + pw * 4 + kq;
-          id[s] = j < it.n ? __ldg(it.ids + j) : -1;
-        }
-        const uint32_t stage = g % kNst;
-        if (!mbar_wait(bar(EMPTY + stage), ((g / kNst) & 1) ^ 1, p.limit_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint32_t dst = sRing + stage * kTileBytes;
+      for (int kt = 0; kt < kMaxTiles; ++kt)
+        if (kt < cur_nt && ok) ok = tile(Kb, ids[kt], kt == 0);
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int r = s * 16 + pw * 4 + kq;
-          const bool valid = id[s] >= 0 && id[s] < it.row_limit;
-          const __nv_bfloat16* row = src + static_cast<int64_t>(valid ? id[s] : 0) * kD + l8 * 8;
-          const uint32_t d = dst + r * 128 + ((l8 ^ (r & 7)) << 4);
-          cp_async16(d, row, valid ? 16u : 0u);
-          cp_async16(d + kKeys * 128, row + 64, valid ? 16u : 0u);
-        }
-        cp_async_commit();
-        if (u > 0) {
-          // the previous tile (and, after the first, Q) has landed
-          cp_async_wait<1>();
-          fence_proxy_async();
-          mbar_arrive(bar(FULL + prev_stage));
-          if (u == 1) mbar_arrive(bar(Q_FULL));
-        }
-        prev_stage = stage;
-        ++g;
-      }
-      if (!ok) break;
-      cp_async_wait<0>();
-      fence_proxy_async();
-      mbar_arrive(bar(FULL + prev_stage));
+      for (int kt = 0; kt < kMaxTiles; ++kt)
+        if (kt < cur_nt && ok) ok = tile(Vb, ids[kt], false);
       ++ait;
+#pragma unroll
+      for (int kt = 0; kt < kMaxTiles; ++kt) ids[kt] = nids[kt];
+      cur = nxt;
+      cur_nt = nxt_nt;
+      have = have_nxt;
     }
-    cp_async_wait<0>();
+    cp_async_wait_all();
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -435,13 +458,20 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
       float mx[kN];
 #pragma unroll
       for (int h = 0; h < kN; ++h) mx[h] = -INFINITY;
-      for (int i = 0; i < nt; ++i) {
-        uint32_t v[16];
-        tmem_ld16(tl + i * kN, v);
-        tmem_wait16(v);
+      for (int i = 0; i < nt; i += 2) {  // two tiles' loads per wait
+        uint32_t v0[16], v1[16];
+        const bool two = i + 1 < nt;
+        tmem_ld16(tl + i * kN, v0);
+        if (two) tmem_ld16(tl + (i + 1) * kN, v1);
+        tmem_wait16(v0);
+        tmem_wait16(v1);
         if ((vmask >> i) & 1u) {
 #pragma unroll
-          for (int h = 0; h < kN; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(v[h]) * p.scale_log2);
+          for (int h = 0; h < kN; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(v0[h]) * p.scale_log2);
+        }
+        if (two && ((vmask >> (i + 1)) & 1u)) {
+#pragma unroll
+          for (int h = 0; h < kN; ++h) mx[h] = fmaxf(mx[h], __uint_as_float(v1[h]) * p.scale_log2);
         }
       }
       {
@@ -464,15 +494,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
       float sum[kN];
 #pragma unroll
       for (int h = 0; h < kN; ++h) sum[h] = 0.0f;
-      for (int i = 0; i < nt; ++i) {
-        const uint32_t slot = pc % kNp;
-        if (!mbar_wait(bar(P_EMPTY + slot), ((pc / kNp) & 1) ^ 1, p.limit_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
-        uint32_t v[16];
-        tmem_ld16(tl + i * kN, v);
-        tmem_wait16(v);
+      // Tile i goes to P slot (pc + i) % kNp.
+      auto emit = [&](int i, uint32_t (&v)[16]) -> bool {
+        const uint32_t t = pc + i, slot = t % kNp;
+        if (!mbar_wait(bar(P_EMPTY + slot), ((t / kNp) & 1) ^ 1, p.limit_ns, abort_flag))
+          return false;
         const bool valid = (vmask >> i) & 1u;
         float pr[kN];
 #pragma unroll
@@ -493,8 +519,19 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(bar(P_FULL + slot));
-        ++pc;
+        return true;
+      };
+      for (int i = 0; i < nt; ++i) {
+        uint32_t v[16];
+        tmem_ld16(tl + i * kN, v);
+        tmem_wait16(v);
+        if (!emit(i, v)) {
+          ok = false;
+          break;
+        }
       }
+      if (!ok) break;
+      pc += nt;
       if (!ok) break;
       {
         const float s = warp_reduce16(sum, lane, [](float a, float b) { return a + b; });
