@@ -184,6 +184,17 @@ dsa_status dsa_stage_times(double* ms, int64_t* launches, int n);
 dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
 
 /*
+ * dsa_debug_force_fallback — test hook for the exact fallback of the select
+ * stage.  With period > 0, every later dsa_prefill call sends each query row
+ * t with t % period == 0 to the fallback (scores recomputed for the whole
+ * row and selected exactly), whatever its candidate list holds; period = 0
+ * restores the normal behaviour.  The results are the same either way; only
+ * the path and the time differ.  Process-wide setting, not thread-safe.
+ * Returns DSA_ERR_INVALID_ARG for period < 0.
+ */
+dsa_status dsa_debug_force_fallback(int period);
+
+/*
  * dsa_decode_static — dsa_decode for callers that cannot allocate device
  * memory: a plugin whose host application owns every device allocation, or
  * a serving loop that must not call cudaMalloc (it can synchronise the device

@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "DsaError", "load", "dsa_version", "dsa_status_string", "dsa_indexer_scores",
     "dsa_prefill_workspace_size", "dsa_prefill", "dsa_decode_workspace_size", "dsa_decode",
-    "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "IDX_FP8_E4M3", "IDX_BF16",
+    "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "dsa_debug_force_fallback", "IDX_FP8_E4M3", "IDX_BF16",
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
 ]
 
@@ -56,6 +56,7 @@ def load() -> ctypes.CDLL:
         "dsa_sync_status": ([P], I),
         "dsa_last_stats": ([P, ctypes.POINTER(ctypes.c_int64), P], I),
         "dsa_debug_wait_timeout": ([ctypes.c_uint64, P], I),
+        "dsa_debug_force_fallback": ([I], I),
         "dsa_decode_static": ([P, P, P, P, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P], I),
         "dsa_stage_timing": ([I], I),
         "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
@@ -218,6 +219,12 @@ def dsa_last_stats(workspace: torch.Tensor, stream=None) -> dict:
     out = (ctypes.c_int64 * 4)()
     _check(load().dsa_last_stats(_dev(workspace, "workspace"), out, _stream(stream)), "dsa_last_stats")
     return {"fallback_rows": out[0], "overflow_rows": out[1], "candidates": out[2]}
+
+
+def dsa_debug_force_fallback(period: int) -> None:
+    """Send every prefill row t with t % period == 0 to the select's exact
+    fallback (period 0: off).  Test hook; results are unchanged."""
+    _check(load().dsa_debug_force_fallback(int(period)), "dsa_debug_force_fallback")
 
 
 def dsa_debug_wait_timeout(limit_ns: int, stream=None) -> None:

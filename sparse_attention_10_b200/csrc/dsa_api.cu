@@ -9,6 +9,7 @@
 //   5. attn_kernel            gathered sparse MQA attention.
 // dsa_decode runs the scan, the per-sequence select and split attention.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -20,6 +21,9 @@
 namespace dsa {
 
 __device__ unsigned int g_status = 0;
+
+// dsa_debug_force_fallback's period (0: off).
+std::atomic<int> g_force_fb_period{0};
 
 namespace {
 
@@ -53,12 +57,17 @@ struct PrefillPlan {
   int target;       // candidates aimed for per row by the threshold
   int samp_ld;
   int fb_ctas;
-  size_t off_counters, off_tau, off_cand_n, off_cand, off_samp, off_fb_rows, off_fb_scratch, total;
+  size_t off_counters, off_tau, off_cand_n, off_cand, off_samp, off_fb_rows, off_fb_scratch,
+      off_fb_hist, off_fb_slow, total;
 };
 
 PrefillPlan plan_prefill(int64_t L, int top_k) {
   PrefillPlan p{};
-  p.target = (top_k * 17 + 9) / 10;                      // 1.7 k
+  // 1.4 k: on the synthetic workloads the realized count has a spread of
+  // about 0.1 k around the target, so fewer than k survivors (a fallback
+  // row) is a > 4-sigma event; each extra 0.1 k costs filter stores and
+  // select work in proportion.
+  p.target = (top_k * 7 + 2) / 5;
   p.cap_half = ((top_k * 5 / 4 + 128) + 15) / 16 * 16;    // per half: 1.25 k + 128
   p.cap_all = p.cap_half;  // rows kept whole must fit one column half
   p.samp_ld = kSampTilesMax * kBN;
@@ -78,6 +87,10 @@ PrefillPlan plan_prefill(int64_t L, int top_k) {
   o = align_up(o + L * sizeof(int));
   p.off_fb_scratch = o;
   o = align_up(o + static_cast<size_t>(p.fb_ctas) * L * sizeof(unsigned long long));
+  p.off_fb_hist = o;
+  o = align_up(o + static_cast<size_t>(p.fb_ctas) * 4096 * sizeof(unsigned int));
+  p.off_fb_slow = o;
+  o = align_up(o + static_cast<size_t>(p.fb_ctas) * sizeof(int));
   p.total = o;
   return p;
 }
@@ -313,9 +326,12 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   sl.d = d_idx;
   sl.scale = iscale;
   sl.fb_scratch = fb_scratch;
+  sl.fb_hist = reinterpret_cast<unsigned int*>(ws + plan.off_fb_hist);
+  sl.fb_slow = reinterpret_cast<int*>(ws + plan.off_fb_slow);
   sl.fb_ctas = plan.fb_ctas;
+  sl.force_fb_period = g_force_fb_period.load();
   {
-    StageScope scope(3, 2, s);
+    StageScope scope(3, 4, s);
     if ((st = launch_select(sl, s)) != DSA_OK) return st;
   }
 
@@ -463,6 +479,12 @@ dsa_status dsa_stage_times(double* ms, int64_t* launches, int n) {
     g_launches[i] = 0;
   }
   return st;
+}
+
+dsa_status dsa_debug_force_fallback(int period) {
+  if (period < 0) return DSA_ERR_INVALID_ARG;
+  dsa::g_force_fb_period.store(period);
+  return DSA_OK;
 }
 
 dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream) {

@@ -56,14 +56,18 @@ struct SelectLaunch {
   const float* tau;      // per-row threshold (zero-mode rows are marked by its bits)
   int32_t* indices;
   int* fb_rows;          // [L] rows that need the exact fallback
-  int* counters;         // [0] fallback rows, [1] overflow rows, [2] candidates
+  int force_fb_period;   // > 0: rows t % period == 0 go to the fallback (test hook)
+  int* counters;         // [0] fallback rows, [1] overflow rows, [2] candidates,
+                         // [3] fallback rows left to the one-CTA path
   // fallback inputs
   const void* q_idx;
   const void* k_idx;
   int esize, d;
   float scale;
   unsigned long long* fb_scratch;  // [fb_ctas, L]
-  int fb_ctas;
+  unsigned int* fb_hist;           // [fb_ctas, 4096]
+  int* fb_slow;                    // [fb_ctas]
+  int fb_ctas;                     // fallback rows handled by the grid-wide path
 };
 
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream);

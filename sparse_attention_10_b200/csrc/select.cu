@@ -31,6 +31,8 @@ namespace dsa {
 namespace {
 
 constexpr int kSelThreads = 256;
+constexpr int kFbBins = 4096;   // fallback histogram: bits 19..30 of a non-negative score word
+constexpr int kFbChunk = 4096;  // keys per scoring work item
 constexpr uint32_t kZeroModeTauBits = 1u;  // tau of a row whose threshold is "score > 0"
 
 __device__ __forceinline__ void block_find_from_top(const unsigned int* hist, int R, int* out) {
@@ -193,56 +195,60 @@ struct SelParams {
   int32_t* indices;
   int* fb_rows;
   int* counters;
+  int force_fb_period;
 };
 
-__global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
-  extern __shared__ unsigned long long sel_smem[];
-  // raw: the row's two candidate lists (64-bit keys); after the merge the same
-  // bytes hold the second score buffer and both position buffers.
-  unsigned long long* raw = sel_smem;                                    // [kSortCap]
-  uint32_t* sc1 = reinterpret_cast<uint32_t*>(raw);                      // [kSortCap]
-  uint16_t* ps0 = reinterpret_cast<uint16_t*>(sc1 + kSortCap);           // [kSortCap]
-  uint16_t* ps1 = ps0 + kSortCap;                                        // [kSortCap]
-  uint32_t* sc0 = reinterpret_cast<uint32_t*>(raw + kSortCap);           // [kSortCap]
-  uint32_t* ix = sc0 + kSortCap;                                         // [kSortCap]
-  uint32_t* cnt = ix + kSortCap;                                         // [warps][256] / bitmap
-  uint32_t* base = cnt + kSortWarps * 256;                               // [256]
-  uint32_t* misc = base + 256;                                           // [8]
-  // (positions of the merged run fit 16 bits: n <= kSortCap < 65536)
+struct SelSmem {
+  unsigned long long* raw;  // [kSortCap] candidate keys; after the merge the same bytes
+  uint32_t* sc1;            //   hold sc1 [kSortCap], ps0 [kSortCap], ps1 [kSortCap]
+  uint16_t* ps0;
+  uint16_t* ps1;
+  uint32_t* sc0;            // [kSortCap] score words
+  uint32_t* ix;             // [kSortCap] key indices
+  uint32_t* cnt;            // [warps][256] / bitmap
+  uint32_t* base;           // [256]
+  uint32_t* misc;           // [8]
+};
+constexpr size_t kSelSmemBytes =
+    static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
+
+__device__ __forceinline__ SelSmem carve_sel_smem(unsigned long long* smem) {
+  SelSmem sm;
+  sm.raw = smem;
+  sm.sc1 = reinterpret_cast<uint32_t*>(smem);
+  sm.ps0 = reinterpret_cast<uint16_t*>(sm.sc1 + kSortCap);
+  sm.ps1 = sm.ps0 + kSortCap;
+  sm.sc0 = reinterpret_cast<uint32_t*>(smem + kSortCap);
+  sm.ix = sm.sc0 + kSortCap;
+  sm.cnt = sm.ix + kSortCap;
+  sm.base = sm.cnt + kSortWarps * 256;
+  sm.misc = sm.base + 256;
+  return sm;
+}
+
+// The n kept candidates of row t (score words sc0 and key indices ix, in
+// ascending index order; n <= kSortCap) are sorted by score, descending and
+// stable, and the first m key indices are written to out, padded with -1 up
+// to top_k.  zero_mode: every positive score of the row is among the
+// candidates and the zeros are ranked by index.  Every thread calls.
+__device__ void sort_emit(const SelSmem& sm, int n, int m, bool zero_mode, int64_t t, int top_k,
+                          int32_t* out) {
+  uint32_t* sc0 = sm.sc0;
+  uint32_t* sc1 = sm.sc1;
+  uint16_t* ps0 = sm.ps0;
+  uint16_t* ps1 = sm.ps1;
+  uint32_t* ix = sm.ix;
+  uint32_t* cnt = sm.cnt;
+  uint32_t* base = sm.base;
+  uint32_t* misc = sm.misc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
-    const int m = static_cast<int>(min64(p.top_k, t + 1));
-    const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
-    const bool overflow = n0 > p.cap || n1 > p.cap || n0 + n1 > kSortCap;
-    const bool zero_mode = __float_as_uint(p.tau[t]) == kZeroModeTauBits;
-    const int n = n0 + n1;
-    if (overflow || (!zero_mode && n < m)) {
-      if (threadIdx.x == 0) {
-        const int pos = atomicAdd(&p.counters[0], 1);
-        p.fb_rows[pos] = static_cast<int>(t);
-        if (overflow) atomicAdd(&p.counters[1], 1);
-      }
-      continue;
-    }
-    if (threadIdx.x == 0) {
-      atomicAdd(&p.counters[2], n);
-      misc[0] = 0u;           // OR of (score word - row minimum)
-      misc[1] = 0xFFFFFFFFu;  // AND of the same
-      misc[2] = 0u;           // positive scores
-      misc[3] = 0xFFFFFFFFu;  // row minimum score word
-    }
-    const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
-    const unsigned long long* c1 = c0 + p.cap;
-    // Both lists in flight at once (8-byte asynchronous copies), one wait.
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const unsigned long long* src = i < n0 ? c0 + i : c1 + (i - n0);
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(raw + i)), "l"(src)
-                   : "memory");
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
-    merge_by_index(raw, n0, raw + n0, n1, p.scale, sc0, ix);
-    __syncthreads();
+  if (threadIdx.x == 0) {
+    misc[0] = 0u;           // OR of (score word - row minimum)
+    misc[1] = 0xFFFFFFFFu;  // AND of the same
+    misc[2] = 0u;           // positive scores
+    misc[3] = 0xFFFFFFFFu;  // row minimum score word
+  }
+  __syncthreads();
     // Score words of non-negative floats order like the values; subtracting
     // the row minimum keeps the order and leaves fewer bytes to sort.
     uint32_t lo = 0xFFFFFFFFu, pos = 0u;
@@ -278,9 +284,8 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     uint32_t* ks = sc0;
     uint16_t* ps = nullptr;
     stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary, cnt, base);
-    int32_t* out = p.indices + t * p.top_k;
     if (!zero_mode || npos >= m) {
-      for (int i = threadIdx.x; i < p.top_k; i += blockDim.x)
+      for (int i = threadIdx.x; i < top_k; i += blockDim.x)
         out[i] = i < m ? static_cast<int32_t>(ix[ps ? ps[i] : i]) : -1;
     } else {
       // Every positive score is a candidate; the rest of the row ranks the
@@ -328,8 +333,43 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
           ++rank;
         }
       }
-      for (int i = m + threadIdx.x; i < p.top_k; i += blockDim.x) out[i] = -1;
+      for (int i = m + threadIdx.x; i < top_k; i += blockDim.x) out[i] = -1;
     }
+}
+
+__global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
+  extern __shared__ unsigned long long sel_smem[];
+  const SelSmem sm = carve_sel_smem(sel_smem);
+  unsigned long long* raw = sm.raw;
+  for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
+    const int m = static_cast<int>(min64(p.top_k, t + 1));
+    const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
+    const bool overflow = n0 > p.cap || n1 > p.cap || n0 + n1 > kSortCap;
+    const bool zero_mode = __float_as_uint(p.tau[t]) == kZeroModeTauBits;
+    const int n = n0 + n1;
+    const bool forced = p.force_fb_period > 0 && t % p.force_fb_period == 0;
+    if (overflow || forced || (!zero_mode && n < m)) {
+      if (threadIdx.x == 0) {
+        const int pos = atomicAdd(&p.counters[0], 1);
+        p.fb_rows[pos] = static_cast<int>(t);
+        if (overflow) atomicAdd(&p.counters[1], 1);
+      }
+      continue;
+    }
+    if (threadIdx.x == 0) atomicAdd(&p.counters[2], n);
+    const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
+    const unsigned long long* c1 = c0 + p.cap;
+    // Both lists in flight at once (8-byte asynchronous copies), one wait.
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const unsigned long long* src = i < n0 ? c0 + i : c1 + (i - n0);
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(raw + i)), "l"(src)
+                   : "memory");
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    merge_by_index(raw, n0, raw + n0, n1, p.scale, sm.sc0, sm.ix);
+    __syncthreads();
+    sort_emit(sm, n, m, zero_mode, t, p.top_k, p.indices + t * p.top_k);
     __syncthreads();
   }
 }
@@ -342,9 +382,12 @@ struct FbParams {
   int esize, d;
   float scale;
   const int* fb_rows;
-  const int* counters;
+  int* counters;                 // [0] fallback rows, [3] rows left to the one-CTA path
   int32_t* indices;
-  unsigned long long* scratch;   // [gridDim.x, L]
+  unsigned long long* scratch;   // [slots, L]: keys of fallback row f (f < slots) / of a CTA
+  unsigned int* hist;            // [slots, kFbBins]
+  int* slow;                     // [slots] fallback slots left to the one-CTA path
+  int slots;
 };
 
 template <int ESIZE>
@@ -406,6 +449,149 @@ __device__ __forceinline__ float dot_row(const float* q, const void* base, int64
   return acc[0];
 }
 
+// Scores of fallback rows f < slots, spread over the whole grid: work item
+// (f, c) computes keys c * kFbChunk .. +kFbChunk of row fb_rows[f] as 64-bit
+// keys (score word << 32 | ~s) into scratch[f] and adds them to the row's
+// histogram of score bits 19..30.
+template <int ESIZE>
+__global__ void __launch_bounds__(kSelThreads) fb_score_kernel(const FbParams p) {
+  __shared__ float qf[DSA_MAX_INDEX_DIM];
+  __shared__ unsigned int h[kFbBins];
+  const int lane = threadIdx.x & 31;
+  const int nf = min(*(volatile const int*)p.counters, p.slots);
+  const int cpr = static_cast<int>((p.L + kFbChunk - 1) / kFbChunk);
+  const int64_t items = static_cast<int64_t>(nf) * cpr;
+  for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
+    const int f = static_cast<int>(item / cpr), c = static_cast<int>(item % cpr);
+    const int64_t t = p.fb_rows[f];
+    const int64_t s0 = static_cast<int64_t>(c) * kFbChunk;
+    if (s0 > t) continue;
+    const int64_t s1 = min64(t + 1, s0 + kFbChunk);
+    load_row_f32<ESIZE>(p.q_idx, t, p.d, qf);
+    for (int i = threadIdx.x; i < kFbBins; i += blockDim.x) h[i] = 0u;
+    __syncthreads();
+    unsigned long long* out = p.scratch + static_cast<int64_t>(f) * p.L;
+    for (int64_t s = s0 + threadIdx.x; s < s0 + kFbChunk; s += blockDim.x) {
+      const bool ok = s < s1;
+      uint32_t bits = 0u;
+      if (ok) {
+        const float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, s, p.d), p.scale);
+        bits = sc > 0.0f ? __float_as_uint(sc) : 0u;
+        out[s] = (static_cast<unsigned long long>(bits) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(s));
+      }
+      // ReLU zeros are common: one add per warp for them
+      const uint32_t zeros = __ballot_sync(0xFFFFFFFFu, ok && bits == 0u);
+      if (lane == 0 && zeros) atomicAdd(&h[0], static_cast<unsigned int>(__popc(zeros)));
+      if (ok && bits != 0u) atomicAdd(&h[bits >> 19], 1u);
+    }
+    __syncthreads();
+    unsigned int* gh = p.hist + static_cast<int64_t>(f) * kFbBins;
+    for (int i = threadIdx.x; i < kFbBins; i += blockDim.x)
+      if (h[i]) atomicAdd(&gh[i], h[i]);
+    __syncthreads();
+  }
+}
+
+// Select of fallback rows f < slots from their scored keys: the histogram
+// gives the bin b holding the m-th largest score; the keys in bins >= b are
+// compacted in ascending index order into shared memory and go through the
+// same sort as the candidates of the main select.  Rows whose keys in bins
+// >= b do not fit (b = 0, where the ReLU zeros are) are left to the one-CTA
+// path.
+__global__ void __launch_bounds__(kSortThreads, 1) fb_select_kernel(const FbParams p) {
+  extern __shared__ unsigned long long sel_smem[];
+  const SelSmem sm = carve_sel_smem(sel_smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* wsum = sm.base;   // [kSortWarps] per-warp counts, then the scan
+  uint32_t* misc = sm.misc;
+  const int nf = min(*(volatile const int*)p.counters, p.slots);
+  constexpr int kPer = kFbBins / kSortThreads;  // bins per thread
+  static_assert(kPer * kSortThreads == kFbBins, "bins per thread");
+  for (int f = blockIdx.x; f < nf; f += gridDim.x) {
+    const int64_t t = p.fb_rows[f];
+    const int n = static_cast<int>(t + 1);
+    const int m = min(p.top_k, n);
+    const unsigned int* gh = p.hist + static_cast<int64_t>(f) * kFbBins;
+    // thread i owns bins kFbBins-1-kPer*i .. kFbBins-kPer*(i+1) (descending)
+    unsigned int loc = 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) loc += gh[kFbBins - 1 - kPer * threadIdx.x - q];
+    unsigned int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    if (threadIdx.x == 0) misc[4] = 0xFFFFFFFFu;
+    __syncthreads();
+    unsigned int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    const unsigned int ex = before + incl - loc;  // count in bins above my range
+    if (ex < static_cast<unsigned int>(m) && ex + loc >= static_cast<unsigned int>(m)) {
+      unsigned int run = ex;
+      for (int q = 0; q < kPer; ++q) {
+        const int b = kFbBins - 1 - kPer * threadIdx.x - q;
+        if (run + gh[b] >= static_cast<unsigned int>(m)) {
+          misc[4] = static_cast<uint32_t>(b);
+          misc[5] = run + gh[b];  // keys in bins >= b
+          break;
+        }
+        run += gh[b];
+      }
+    }
+    __syncthreads();
+    const uint32_t b = misc[4];
+    const uint32_t total = misc[5];
+    __syncthreads();
+    if (b == 0xFFFFFFFFu || b == 0u || total > static_cast<uint32_t>(kSortCap)) {
+      if (threadIdx.x == 0) p.slow[atomicAdd(&p.counters[3], 1)] = f;
+      continue;
+    }
+    // stable compaction of the keys in bins >= b, four consecutive keys per thread
+    const unsigned long long* keys = p.scratch + static_cast<int64_t>(f) * p.L;
+    uint32_t done = 0;
+    for (int s0 = 0; s0 < n; s0 += 4 * kSortThreads) {
+      const int sb = s0 + 4 * threadIdx.x;
+      unsigned long long k4[4];
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        k4[q] = sb + q < n ? keys[sb + q] : 0ull;
+        c += (sb + q < n && static_cast<uint32_t>(k4[q] >> 51) >= b) ? 1 : 0;
+      }
+      int ic = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, ic, o);
+        if (lane >= o) ic += y;
+      }
+      if (lane == 31) wsum[warp] = static_cast<uint32_t>(ic);
+      __syncthreads();
+      uint32_t pos = done;
+      for (int w = 0; w < warp; ++w) pos += wsum[w];
+      uint32_t all = 0;
+      for (int w = 0; w < kSortWarps; ++w) all += wsum[w];
+      pos += static_cast<uint32_t>(ic - c);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (sb + q < n && static_cast<uint32_t>(k4[q] >> 51) >= b) {
+          sm.sc0[pos] = static_cast<uint32_t>(k4[q] >> 32);
+          sm.ix[pos] = static_cast<uint32_t>(sb + q);
+          ++pos;
+        }
+      }
+      done += all;
+      __syncthreads();
+    }
+    sort_emit(sm, static_cast<int>(total), m, false, t, p.top_k, p.indices + t * p.top_k);
+    __syncthreads();
+  }
+}
+
+// One CTA per row, scores recomputed into the CTA's own scratch row: the
+// fallback slots the shared-memory select left (p.slow) and the fallback
+// rows beyond the slots.
 template <int ESIZE>
 __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p) {
   extern __shared__ unsigned long long fb_smem[];
@@ -415,7 +601,10 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
   float* qf = reinterpret_cast<float*>(shared2 + 4);                   // [d]
   unsigned long long* scratch = p.scratch + static_cast<int64_t>(blockIdx.x) * p.L;
   const int nfb = *(volatile const int*)p.counters;
-  for (int f = blockIdx.x; f < nfb; f += gridDim.x) {
+  const int nslow = *(volatile const int*)(p.counters + 3);
+  const int extra = max(0, nfb - p.slots);
+  for (int w = blockIdx.x; w < nslow + extra; w += gridDim.x) {
+    const int f = w < nslow ? p.slow[w] : p.slots + (w - nslow);
     const int64_t t = p.fb_rows[f];
     const int n = static_cast<int>(t + 1);
     const int m = min(p.top_k, n);
@@ -437,17 +626,31 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
   if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
-  SelParams p{a.L, a.top_k, a.cap, a.scale, a.cand, a.cand_n, a.tau, a.indices, a.fb_rows, a.counters};
-  const size_t smem = static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
+  SelParams p{a.L,      a.top_k,   a.cap,     a.scale,    a.cand,
+              a.cand_n, a.tau,     a.indices, a.fb_rows,  a.counters, a.force_fb_period};
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                                       static_cast<int>(kSelSmemBytes));
   if (e != cudaSuccess) return DSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<int64_t>(a.L, 2 * num_sms()));
-  select_kernel<<<grid, kSortThreads, smem, stream>>>(p);
+  select_kernel<<<grid, kSortThreads, kSelSmemBytes, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
 
-  FbParams f{a.L, a.top_k, a.q_idx, a.k_idx, a.esize, a.d, a.scale, a.fb_rows, a.counters,
-             a.indices, a.fb_scratch};
+  // Fallback rows (their number is known on the device only): scores on the
+  // whole grid, select in shared memory, the rest on one CTA per row.  The
+  // histograms start from zero.
+  if (cudaMemsetAsync(a.fb_hist, 0, static_cast<size_t>(a.fb_ctas) * kFbBins * sizeof(unsigned int),
+                      stream) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  FbParams f{a.L,       a.top_k,      a.q_idx,   a.k_idx,   a.esize,  a.d,     a.scale,
+             a.fb_rows, a.counters,   a.indices, a.fb_scratch, a.fb_hist, a.fb_slow, a.fb_ctas};
+  if (a.esize == 1)
+    fb_score_kernel<1><<<4 * num_sms(), kSelThreads, 0, stream>>>(f);
+  else
+    fb_score_kernel<2><<<4 * num_sms(), kSelThreads, 0, stream>>>(f);
+  e = cudaFuncSetAttribute(fb_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kSelSmemBytes));
+  if (e != cudaSuccess) return DSA_ERR_CUDA;
+  fb_select_kernel<<<a.fb_ctas, kSortThreads, kSelSmemBytes, stream>>>(f);
   const size_t fsmem = static_cast<size_t>(P) * 8 + 256 * 4 + 16 + a.d * 4;
   if (a.esize == 1) {
     e = cudaFuncSetAttribute(fallback_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,

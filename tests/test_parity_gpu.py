@@ -158,6 +158,47 @@ def test_prefill_all_zero_scores(dsa):
     compare(x, "fp8", 256, idx, O, rows=np.array([0, 1, 300, 1000, 2499]))
 
 
+# ------------------------------------------------------------------ exact fallback of the select
+
+@pytest.fixture
+def force_fallback(dsa):
+    yield dsa.dsa_debug_force_fallback
+    dsa.dsa_debug_force_fallback(0)
+
+
+def test_prefill_forced_fallback_many_rows(dsa, force_fallback):
+    # Every 7th row through the fallback: more rows than the grid-wide slots
+    # (one per SM), so the shared-memory select and the one-CTA path both run.
+    x = small_inputs(3000, 96, 4, 128, seed=12)
+    force_fallback(7)
+    idx, O, stats = run_prefill(dsa, x, 256)
+    assert stats["fallback_rows"] == len(range(0, 3000, 7)), stats
+    compare(x, "fp8", 256, idx, O)
+
+
+def test_prefill_forced_fallback_zero_ties(dsa, force_fallback):
+    # All scores zero: the boundary bin is the ReLU zeros', the shared-memory
+    # select declines and the one-CTA path ranks the ties by index.
+    x = small_inputs(1200, 128, 4, 64, seed=13)
+    x["q_idx"] = np.zeros_like(x["q_idx"])
+    force_fallback(5)
+    idx, O, stats = run_prefill(dsa, x, 128)
+    assert stats["fallback_rows"] == len(range(0, 1200, 5)), stats
+    for t in (0, 5, 130, 1195):
+        m = min(128, t + 1)
+        assert idx[t, :m].tolist() == list(range(m))
+    compare(x, "fp8", 128, idx, O, rows=np.array([0, 5, 10, 127, 130, 600, 1195, 1199]))
+
+
+def test_prefill_forced_fallback_bf16_long_rows(dsa, force_fallback):
+    # BF16 index rows of 160, top_k 2048, rows spanning several scoring chunks.
+    x = small_inputs(9000, 160, 16, 128, idx_dtype="bf16", seed=14)
+    force_fallback(1000)
+    idx, O, stats = run_prefill(dsa, x, 2048)
+    assert stats["fallback_rows"] == 9, stats
+    compare(x, "bf16", 2048, idx, O, rows=np.array([0, 1000, 2000, 2047, 4000, 7000, 8000, 8999]))
+
+
 def test_prefill_top_k_2048_small(dsa):
     x = small_inputs(5000, 128, 16, 128, seed=10)
     idx, O, _ = run_prefill(dsa, x, 2048)
