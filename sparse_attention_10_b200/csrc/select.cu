@@ -158,10 +158,11 @@ __device__ __forceinline__ uint32_t key_index(unsigned long long k) {
 }
 
 // Merge two ascending-index runs a[0, na) and b[0, nb) (64-bit candidate
-// keys) into one ascending-index run, written as score words `sc` and key
-// indices `ix` (merge path: each thread finds its split by binary search).
+// keys) into one ascending-index run, written as relu(accumulator) words `sc`
+// and key indices `ix` (merge path: each thread finds its split by binary
+// search).
 __device__ void merge_by_index(const unsigned long long* a, int na, const unsigned long long* b,
-                               int nb, float scale, uint32_t* sc, uint32_t* ix) {
+                               int nb, uint32_t* sc, uint32_t* ix) {
   const int n = na + nb;
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int p0 = min(n, static_cast<int>(threadIdx.x) * per), p1 = min(n, p0 + per);
@@ -178,9 +179,9 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
   for (int p = p0; p < p1; ++p) {
     const bool take_a = j >= nb || (i < na && key_index(a[i]) < key_index(b[j]));
     const unsigned long long k = take_a ? a[i++] : b[j++];
-    // the filter stored the raw accumulator: score = relu(fp32(acc) * scale)
-    const float score = __fmul_rn(__uint_as_float(static_cast<uint32_t>(k >> 32)), scale);
-    sc[p] = score > 0.0f ? __float_as_uint(score) : 0u;
+    // the filter stored the raw accumulator; the sort key starts as relu(acc)
+    const uint32_t acc = static_cast<uint32_t>(k >> 32);
+    sc[p] = __uint_as_float(acc) > 0.0f ? acc : 0u;
     ix[p] = key_index(k);
   }
 }
@@ -341,6 +342,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
   extern __shared__ unsigned long long sel_smem[];
   const SelSmem sm = carve_sel_smem(sel_smem);
   unsigned long long* raw = sm.raw;
+  const int lane = threadIdx.x & 31;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
     const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
@@ -367,8 +369,53 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    merge_by_index(raw, n0, raw + n0, n1, p.scale, sm.sc0, sm.ix);
+    if (threadIdx.x == 0) {
+      sm.misc[4] = 0u;           // largest exponent field of a positive accumulator
+      sm.misc[5] = 0xFFFFFFFFu;  // lowest set bit (exponent of 2) over them, biased by 150
+    }
+    merge_by_index(raw, n0, raw + n0, n1, sm.sc0, sm.ix);
     __syncthreads();
+    // Ordering by relu(acc) is ordering by score = relu(fp32(acc) * scale), ties
+    // included, when the scale is positive and no two distinct accumulators of
+    // the row round to the same score: so when every positive accumulator is a
+    // normal multiple of 4 ulps of the largest one (then the exact products
+    // differ by 2 ulps of the larger score) and the smallest scores stay
+    // normal.  Integer-valued index inputs give that.  Otherwise the keys
+    // become the score words.
+    {
+      uint32_t emax = 0u, pmin = 0xFFFFFFFFu;
+      for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t w = sm.sc0[i];
+        if (w) {
+          const uint32_t e = w >> 23;
+          const uint32_t mant = (w & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+          emax = max(emax, e);
+          pmin = min(pmin, e ? e + static_cast<uint32_t>(__ffs(static_cast<int>(mant)) - 1) : 0u);
+        }
+      }
+      emax = __reduce_max_sync(0xFFFFFFFFu, emax);
+      pmin = __reduce_min_sync(0xFFFFFFFFu, pmin);
+      if (lane == 0) {
+        atomicMax(&sm.misc[4], emax);
+        atomicMin(&sm.misc[5], pmin);
+      }
+      __syncthreads();
+      const uint32_t em = sm.misc[4], pm = sm.misc[5];
+      // every positive accumulator is a multiple of 2^(pm - 150) >= 4 ulps of
+      // the largest (2^(em - 148)); the smallest score, >= 2^(pm - 150) * scale,
+      // is normal
+      const bool by_acc =
+          p.scale > 0.0f &&
+          (pm == 0xFFFFFFFFu ||
+           (pm >= em + 2u && __fmul_rn(ldexpf(1.0f, static_cast<int>(pm) - 150), p.scale) >= 1.17549435e-38f));
+      if (!by_acc) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+          const float sc = __fmul_rn(__uint_as_float(sm.sc0[i]), p.scale);
+          sm.sc0[i] = sc > 0.0f ? __float_as_uint(sc) : 0u;
+        }
+      }
+      __syncthreads();
+    }
     sort_emit(sm, n, m, zero_mode, t, p.top_k, p.indices + t * p.top_k);
     __syncthreads();
   }

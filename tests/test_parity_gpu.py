@@ -148,6 +148,22 @@ def test_prefill_many_ties(dsa):
     compare(x, "fp8", 200, idx, O)
 
 
+def test_prefill_large_accumulators_tie_after_scaling(dsa):
+    # BF16 integers in [244, 256], index dim 256: dot products in [2^23, 2^24)
+    # stay exact in FP32, but with idx_scale 0.55 neighbouring accumulators
+    # round to the same score, so the select must rank by score (ties by
+    # index), not by accumulator.
+    x = small_inputs(1500, 256, 4, 64, idx_dtype="bf16", seed=15)
+    key = synth.stream_key(15, 501, 1500, 256)
+    for name, start in (("q_idx", 0), ("k_idx", 1500 * 256)):
+        v = synth.uniform_ints(key, 1500 * 256, 244, 256, start=start).reshape(1500, 256)
+        x[name] = synth.bf16_bits_of_f32(v.astype(np.float32))   # exact: |v| <= 256
+    idx, O, _ = run_prefill(dsa, x, 64, idx_scale=0.55)
+    ri, ro = oracle.prefill_rows(x, "bf16", 64, idx_scale=0.55)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
 def test_prefill_all_zero_scores(dsa):
     x = small_inputs(2500, 128, 4, 64, seed=9)
     x["q_idx"] = np.zeros_like(x["q_idx"])
