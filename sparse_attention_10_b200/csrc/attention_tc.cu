@@ -538,8 +538,31 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
         if ((lane & 1) == 0) red_sum[(lane >> 1) * 4 + warp] = s;
       }
       mbar_arrive(bar(RED_SUM));
-      if (!mbar_wait(bar(RED_SUM), ait & 1, p.limit_ns, abort_flag) ||
-          !mbar_wait(bar(O_FULL), ait & 1, p.limit_ns, abort_flag)) {
+      if (!mbar_wait(bar(RED_SUM), ait & 1, p.limit_ns, abort_flag)) {
+        ok = false;
+        break;
+      }
+      // Everything but O first: 1 / sum per head in registers and, for split
+      // partials, the (max, sum) words; red_max and red_sum are not read
+      // after TM_EMPTY, whose completion lets the next item overwrite them.
+      float inv[kN];
+#pragma unroll
+      for (int h = 0; h < kN; ++h) {
+        const float4 w = *reinterpret_cast<const float4*>(red_sum + h * 4);
+        const float l = (w.x + w.y) + (w.z + w.w);
+        if (p.nsplit == 1) {
+          inv[h] = l > 0.0f ? 1.0f / l : 0.0f;
+        } else {
+          inv[h] = 1.0f;
+          if (r == 0 && h < p.H) {
+            const float4 m = *reinterpret_cast<const float4*>(red_max + h * 4);
+            float* dst = p.part + ((it.q * p.nsplit + it.sp) * p.H + h) * (kD + 2);
+            dst[0] = fmaxf(fmaxf(m.x, m.y), fmaxf(m.z, m.w));
+            dst[1] = l;
+          }
+        }
+      }
+      if (!mbar_wait(bar(O_FULL), ait & 1, p.limit_ns, abort_flag)) {
         ok = false;
         break;
       }
@@ -547,28 +570,17 @@ __global__ void __launch_bounds__(kThreads, 2) attn_tc_kernel(const TcParams p) 
       uint32_t o[16];
       tmem_ld16(tl, o);
       tmem_wait16(o);
-      // (red_max and red_sum are read before TM_EMPTY: once every thread has
-      // arrived, the next item may overwrite them)
+      tc_fence_before();
+      mbar_arrive(bar(TM_EMPTY));  // O is in registers: the next item's S may start
 #pragma unroll
       for (int h = 0; h < kN; ++h) {
         if (h >= p.H) break;
-        const float4 w = *reinterpret_cast<const float4*>(red_sum + h * 4);
-        const float l = (w.x + w.y) + (w.z + w.w);
-        const float ov = __uint_as_float(o[h]);
-        if (p.nsplit == 1) {
-          p.O[(it.q * p.H + h) * kD + r] = __float2bfloat16_rn(l > 0.0f ? ov / l : 0.0f);
-        } else {
-          float* dst = p.part + ((it.q * p.nsplit + it.sp) * p.H + h) * (kD + 2);
-          dst[2 + r] = ov;
-          if (r == 0) {
-            const float4 m = *reinterpret_cast<const float4*>(red_max + h * 4);
-            dst[0] = fmaxf(fmaxf(m.x, m.y), fmaxf(m.z, m.w));
-            dst[1] = l;
-          }
-        }
+        const float ov = __uint_as_float(o[h]) * inv[h];
+        if (p.nsplit == 1)
+          p.O[(it.q * p.H + h) * kD + r] = __float2bfloat16_rn(ov);
+        else
+          p.part[((it.q * p.nsplit + it.sp) * p.H + h) * (kD + 2) + 2 + r] = ov;
       }
-      tc_fence_before();
-      mbar_arrive(bar(TM_EMPTY));
       ++ait;
     }
   }

@@ -164,6 +164,17 @@ def test_prefill_large_accumulators_tie_after_scaling(dsa):
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
 
 
+def test_prefill_attention_large_norm_key(dsa):
+    # One K row with 64 times the others' norm: queries that keep it get
+    # scores far above the rest, so softmax weights span a wide range.
+    x = small_inputs(1500, 96, 16, 128, seed=16)
+    K = bits_to_f32(x["K"]).reshape(1500, 128)
+    K[7] *= 64.0                              # a power of two: still exact in BF16
+    x["K"] = synth.bf16_bits_of_f32(K)
+    idx, O, _ = run_prefill(dsa, x, 256)
+    compare(x, "fp8", 256, idx, O)
+
+
 def test_prefill_all_zero_scores(dsa):
     x = small_inputs(2500, 128, 4, 64, seed=9)
     x["q_idx"] = np.zeros_like(x["q_idx"])
