@@ -7,15 +7,19 @@
 // per column half of its tile), each in ascending key order.
 //
 // select_kernel: one CTA per row.  The two lists are merged into one
-// ascending-key run; the merge turns each accumulator into the score
-// relu(fp32(acc) * scale) (non-negative, so its bits order like the value).
-// Stable LSD radix passes over the score bytes that differ then order the
-// run by score, descending; equal scores keep ascending key order, so the
-// first min(top_k, t+1) entries are the answer.  Rows whose lists overflowed,
-// or hold fewer keys than needed, are queued for the fallback.
+// ascending-key run of sort keys: relu(acc) when that orders exactly like
+// the score relu(fp32(acc) * scale) (checked per row), else the score word
+// (non-negative, so its bits order like the value).  Stable LSD radix passes
+// over the span of key bits that differ within the row (digits of up to 9
+// bits) then order the run by key, descending; equal keys keep ascending key
+// index, so the first min(top_k, t+1) entries are the answer.  Rows whose
+// lists overflowed, or hold fewer keys than needed, go to the fallback.
 //
-// fallback_kernel: recomputes every causal score of a queued row on CUDA
-// cores (FP32, exact for integer-valued inputs), builds the 64-bit keys
+// Fallback: fb_score_kernel recomputes every causal score of up to one
+// queued row per SM on CUDA cores (FP32, exact for integer-valued inputs)
+// over the whole grid and bins the scores; fb_select_kernel keeps the keys
+// from the bin of the k-th score up and sorts them like select_kernel.
+// fallback_kernel (one CTA per row) takes the rest: it builds the 64-bit keys
 // (score_bits << 32) | (0xFFFFFFFF - s) -- larger key, better rank -- and
 // selects by MSD radix passes plus a bitonic sort of the winners.
 #include <cuda_fp8.h>
@@ -141,11 +145,12 @@ __device__ void finish_row(KeyPtr keys, int n, int m, int top_k, int32_t* out,
 //
 // The filter writes each row's candidates as two lists (one per column half
 // of the indexer tile), each already in ascending key order.  The select
-// merges them into one ascending-index run, then sorts it by score with
-// stable LSD counting passes (descending digit), so equal scores keep
+// merges them into one ascending-index run, then sorts it by key with
+// stable LSD counting passes (descending digit), so equal keys keep
 // ascending index: the result is the (score desc, index asc) order, and the
-// first m entries are the answer.  Only the score bytes that differ within
-// the row get a pass.  Ranks inside a warp come from __match_any_sync, so the
+// first m entries are the answer.  Only the span of key bits that differ
+// within the row is sorted, in digits of up to 9 bits (integer-valued inputs
+// need one pass).  Ranks inside a warp come from __match_any_sync, so the
 // passes use no atomics.
 
 constexpr int kSortThreads = 512;
@@ -206,12 +211,12 @@ struct SelSmem {
   uint16_t* ps1;
   uint32_t* sc0;            // [kSortCap] score words
   uint32_t* ix;             // [kSortCap] key indices
-  uint32_t* cnt;            // [warps][256] / bitmap
-  uint32_t* base;           // [256]
+  uint32_t* cnt;            // [warps][256] words: 16-bit radix counters [warps][512] / bitmap
+  uint32_t* base;           // [512 + warps]
   uint32_t* misc;           // [8]
 };
 constexpr size_t kSelSmemBytes =
-    static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 256 + 8) * 4;
+    static_cast<size_t>(kSortCap) * (8 + 4 + 4) + (kSortWarps * 256 + 512 + kSortWarps + 8) * 4;
 
 __device__ __forceinline__ SelSmem carve_sel_smem(unsigned long long* smem) {
   SelSmem sm;
@@ -223,7 +228,7 @@ __device__ __forceinline__ SelSmem carve_sel_smem(unsigned long long* smem) {
   sm.ix = sm.sc0 + kSortCap;
   sm.cnt = sm.ix + kSortCap;
   sm.base = sm.cnt + kSortWarps * 256;
-  sm.misc = sm.base + 256;
+  sm.misc = sm.base + 512 + kSortWarps;
   return sm;
 }
 
@@ -284,7 +289,8 @@ __device__ void sort_emit(const SelSmem& sm, int n, int m, bool zero_mode, int64
     const int npos = static_cast<int>(misc[2]);
     uint32_t* ks = sc0;
     uint16_t* ps = nullptr;
-    stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary, cnt, base);
+    stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary,
+                                                      reinterpret_cast<uint16_t*>(cnt), base);
     if (!zero_mode || npos >= m) {
       for (int i = threadIdx.x; i < top_k; i += blockDim.x)
         out[i] = i < m ? static_cast<int32_t>(ix[ps ? ps[i] : i]) : -1;

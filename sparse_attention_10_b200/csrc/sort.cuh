@@ -105,76 +105,77 @@ __device__ unsigned long long* stable_sort_by_score(unsigned long long* a, unsig
 
 namespace dsa {
 
-// Stable pass on 32-bit score words with 16-bit payloads (positions):
-// (kout, pout) = (kin, pin) ordered by byte SHIFT/8 of the key, DESCENDING,
-// equal bytes in input order.  pin == nullptr means the identity payload.
-// Same warp/slot/lane ownership and atomic-free ranking as radix_pass_desc.
-template <int WARPS, int SLOTS, int SHIFT>
-__device__ void radix_pass32_desc(const uint32_t* kin, const uint16_t* pin, uint32_t* kout,
-                                  uint16_t* pout, int n, uint32_t* cnt, uint32_t* base) {
+// Stable pass on 32-bit keys with 16-bit payloads (positions):
+// (kout, pout) = (kin, pin) ordered by the `width`-bit digit (key >> shift),
+// width <= 9, DESCENDING, equal digits in input order.  pin == nullptr means
+// the identity payload.  Warp w owns items [w * chunk, (w + 1) * chunk), lane
+// order within each 32-item slot; ranks inside a warp come from
+// __match_any_sync on the digit, so no atomics.  Per-warp digit counters are
+// 16-bit (a warp holds at most 32 * SLOTS items): cnt16 is [WARPS][512],
+// base [512].
+template <int WARPS, int SLOTS>
+__device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint32_t* kout,
+                                 uint16_t* pout, int n, int shift, int width, uint16_t* cnt16,
+                                 uint32_t* base) {
+  constexpr int kBins = 512;
+  static_assert(WARPS * 32 >= kBins, "one thread per digit");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = (n + WARPS * 32 - 1) / (WARPS * 32) * 32;  // items per warp
   const int slots = chunk / 32;
-  uint32_t* wc = cnt + warp * 256;
-  for (int d = lane; d < 256; d += 32) wc[d] = 0;
+  const uint32_t nd = 1u << width, top = nd - 1u;
+  uint16_t* wc = cnt16 + warp * kBins;
+  for (int d = lane; d < kBins; d += 32) wc[d] = 0;
   __syncwarp();
   const uint32_t lt = (1u << lane) - 1u;
-  uint32_t dr[SLOTS];  // digit (bits 16..24, 256 = no item) | rank in warp (bits 0..15)
+  uint32_t dr[SLOTS];  // digit (bits 16..25, 512 = no item) | rank in warp (bits 0..15)
 #pragma unroll
   for (int j = 0; j < SLOTS; ++j) {
     if (j < slots) {
       const int i = warp * chunk + j * 32 + lane;
       const bool ok = i < n;
-      const uint32_t d = ok ? 255u - ((kin[i] >> SHIFT) & 255u) : 256u;
+      const uint32_t d = ok ? top - ((kin[i] >> shift) & top) : 512u;
       const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
       const uint32_t before = ok ? wc[d] : 0u;
       dr[j] = (d << 16) | (before + __popc(peers & lt));
       __syncwarp();
-      if (ok && lane == __ffs(peers) - 1) wc[d] = before + __popc(peers);
+      if (ok && lane == __ffs(peers) - 1) wc[d] = static_cast<uint16_t>(before + __popc(peers));
       __syncwarp();
     }
   }
   __syncthreads();
-  if (threadIdx.x < 256) {  // per digit: warp-exclusive prefix, digit total
-    const int d = threadIdx.x;
-    uint32_t run = 0;
+  // per digit: exclusive prefix over the warps (in place), digit total
+  const int d = threadIdx.x;
+  uint32_t total = 0;
+  if (d < kBins) {
 #pragma unroll 4
     for (int w = 0; w < WARPS; ++w) {
-      const uint32_t c = cnt[w * 256 + d];
-      cnt[w * 256 + d] = run;
-      run += c;
+      const uint32_t c = cnt16[w * kBins + d];
+      cnt16[w * kBins + d] = static_cast<uint16_t>(total);
+      total += c;
     }
-    base[d] = run;
   }
+  // exclusive scan of the digit totals over the block (digits in thread order)
+  uint32_t incl = total;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) base[kBins + warp] = incl;  // warp sums after the digit bases
   __syncthreads();
-  if (threadIdx.x < 32) {  // exclusive scan of the 256 digit totals
-    uint32_t loc[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      loc[q] = base[lane * 8 + q];
-      sum += loc[q];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    uint32_t ex = incl - sum;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      base[lane * 8 + q] = ex;
-      ex += loc[q];
-    }
+  if (d < kBins) {
+    uint32_t off = 0;
+    for (int w = 0; w < warp; ++w) off += base[kBins + w];
+    base[d] = off + incl - total;
   }
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < SLOTS; ++j) {
     if (j < slots) {
-      const uint32_t d = dr[j] >> 16;
-      if (d < 256u) {
+      const uint32_t dg = dr[j] >> 16;
+      if (dg < 512u) {
         const int i = warp * chunk + j * 32 + lane;
-        const uint32_t pos = base[d] + cnt[warp * 256 + d] + (dr[j] & 0xFFFFu);
+        const uint32_t pos = base[dg] + cnt16[warp * kBins + dg] + (dr[j] & 0xFFFFu);
         kout[pos] = kin[i];
         pout[pos] = pin ? pin[i] : static_cast<uint16_t>(i);
       }
@@ -183,33 +184,39 @@ __device__ void radix_pass32_desc(const uint32_t* kin, const uint16_t* pin, uint
   __syncthreads();
 }
 
-// Stable sort of (score word, position) pairs, descending by score, one pass
-// per differing score byte.  Returns through *k / *p the buffers holding the
-// result; p0 == nullptr on entry means positions 0..n-1.
+// Stable sort of (key, position) pairs, descending by key, over the bits that
+// differ among the keys (`vary` = OR ^ AND of the keys): the span from the
+// lowest to the highest differing bit is cut into equal digits of at most 9
+// bits, one pass each, least significant first.  Returns through *k / *p the
+// buffers holding the result; *p == nullptr means no pass ran (input order).
+// cnt16 needs WARPS * 512 16-bit counters, base 512 + WARPS words.
 template <int WARPS, int SLOTS>
 __device__ void stable_sort32_by_score(uint32_t** k, uint16_t** p, uint32_t* k_alt,
                                        uint16_t* p_alt, uint16_t* p_first, int n, uint32_t vary,
-                                       uint32_t* cnt, uint32_t* base) {
+                                       uint16_t* cnt16, uint32_t* base) {
   uint32_t* kc = *k;
   uint16_t* pc = nullptr;             // identity until the first pass
   uint32_t* kn = k_alt;
   uint16_t* pn = p_first;
   uint16_t* spare = p_alt;
-#define DSA_PASS(SH)                                                                  \
-  if ((vary >> SH) & 255u) {                                                          \
-    radix_pass32_desc<WARPS, SLOTS, SH>(kc, pc, kn, pn, n, cnt, base);                \
-    uint32_t* tk = kc;                                                                \
-    kc = kn;                                                                          \
-    kn = tk;                                                                          \
-    uint16_t* tp = pc ? pc : spare;                                                   \
-    pc = pn;                                                                          \
-    pn = tp;                                                                          \
+  if (vary != 0u) {
+    const int lo = __ffs(static_cast<int>(vary)) - 1;
+    const int hi = 31 - __clz(static_cast<int>(vary));
+    const int span = hi - lo + 1;
+    const int passes = (span + 8) / 9;
+    const int width = (span + passes - 1) / passes;
+    for (int q = 0; q < passes; ++q) {
+      const int sh = lo + q * width;
+      const int wd = min(width, hi + 1 - sh);
+      radix_pass32_var<WARPS, SLOTS>(kc, pc, kn, pn, n, sh, wd, cnt16, base);
+      uint32_t* tk = kc;
+      kc = kn;
+      kn = tk;
+      uint16_t* tp = pc ? pc : spare;
+      pc = pn;
+      pn = tp;
+    }
   }
-  DSA_PASS(0)
-  DSA_PASS(8)
-  DSA_PASS(16)
-  DSA_PASS(24)
-#undef DSA_PASS
   *k = kc;
   *p = pc;  // nullptr: no pass ran, order is the input order
 }
