@@ -162,12 +162,56 @@ __device__ __forceinline__ uint32_t key_index(unsigned long long k) {
   return 0xFFFFFFFFu - static_cast<uint32_t>(k);
 }
 
+// Row statistics of the sort keys: minimum, maximum, OR of all keys, number
+// of non-zero keys.  Per-thread partials are combined with warp reductions
+// and shared-memory atomics into misc[0..3], which thread 0 set to
+// (~0, 0, 0, 0) before a barrier; every thread calls, then a barrier.
+struct KeyStats {
+  uint32_t kmin, kmax, kor;
+  int npos;
+};
+
+__device__ __forceinline__ void stats_add(uint32_t w, uint32_t& lo, uint32_t& hi, uint32_t& orr,
+                                          uint32_t& pos) {
+  lo = min(lo, w);
+  hi = max(hi, w);
+  orr |= w;
+  pos += w != 0u;
+}
+
+__device__ __forceinline__ void stats_init(uint32_t* misc) {
+  misc[0] = 0xFFFFFFFFu;
+  misc[1] = 0u;
+  misc[2] = 0u;
+  misc[3] = 0u;
+}
+
+__device__ __forceinline__ void stats_reduce(uint32_t lo, uint32_t hi, uint32_t orr, uint32_t pos,
+                                             uint32_t* misc) {
+  lo = __reduce_min_sync(0xFFFFFFFFu, lo);
+  hi = __reduce_max_sync(0xFFFFFFFFu, hi);
+  orr = __reduce_or_sync(0xFFFFFFFFu, orr);
+  pos = __reduce_add_sync(0xFFFFFFFFu, pos);
+  if ((threadIdx.x & 31) == 0) {
+    atomicMin(&misc[0], lo);
+    atomicMax(&misc[1], hi);
+    atomicOr(&misc[2], orr);
+    atomicAdd(&misc[3], pos);
+  }
+}
+
+__device__ __forceinline__ KeyStats stats_read(const uint32_t* misc) {
+  return KeyStats{misc[0], misc[1], misc[2], static_cast<int>(misc[3])};
+}
+
 // Merge two ascending-index runs a[0, na) and b[0, nb) (64-bit candidate
 // keys) into one ascending-index run, written as relu(accumulator) words `sc`
 // and key indices `ix` (merge path: each thread finds its split by binary
-// search).
+// search); the thread's partial key statistics and, over the positive keys,
+// largest exponent field and lowest set bit are accumulated on the way.
 __device__ void merge_by_index(const unsigned long long* a, int na, const unsigned long long* b,
-                               int nb, uint32_t* sc, uint32_t* ix) {
+                               int nb, uint32_t* sc, uint32_t* ix, uint32_t& klo, uint32_t& khi,
+                               uint32_t& orr, uint32_t& pos, uint32_t& emax, uint32_t& pmin) {
   const int n = na + nb;
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int p0 = min(n, static_cast<int>(threadIdx.x) * per), p1 = min(n, p0 + per);
@@ -186,8 +230,16 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
     const unsigned long long k = take_a ? a[i++] : b[j++];
     // the filter stored the raw accumulator; the sort key starts as relu(acc)
     const uint32_t acc = static_cast<uint32_t>(k >> 32);
-    sc[p] = __uint_as_float(acc) > 0.0f ? acc : 0u;
+    const uint32_t w = __uint_as_float(acc) > 0.0f ? acc : 0u;
+    sc[p] = w;
     ix[p] = key_index(k);
+    stats_add(w, klo, khi, orr, pos);
+    if (w) {  // exponent field and lowest set bit (exponent of 2, biased by 150)
+      const uint32_t e = w >> 23;
+      const uint32_t mant = (w & 0x7FFFFFu) | (e ? 0x800000u : 0u);
+      emax = max(emax, e);
+      pmin = min(pmin, e ? e + static_cast<uint32_t>(__ffs(static_cast<int>(mant)) - 1) : 0u);
+    }
   }
 }
 
@@ -238,7 +290,7 @@ __device__ __forceinline__ SelSmem carve_sel_smem(unsigned long long* smem) {
 // to top_k.  zero_mode: every positive score of the row is among the
 // candidates and the zeros are ranked by index.  Every thread calls.
 __device__ void sort_emit(const SelSmem& sm, int n, int m, bool zero_mode, int64_t t, int top_k,
-                          int32_t* out) {
+                          int32_t* out, const KeyStats& st) {
   uint32_t* sc0 = sm.sc0;
   uint32_t* sc1 = sm.sc1;
   uint16_t* ps0 = sm.ps0;
@@ -246,51 +298,21 @@ __device__ void sort_emit(const SelSmem& sm, int n, int m, bool zero_mode, int64
   uint32_t* ix = sm.ix;
   uint32_t* cnt = sm.cnt;
   uint32_t* base = sm.base;
-  uint32_t* misc = sm.misc;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    misc[0] = 0u;           // OR of (score word - row minimum)
-    misc[1] = 0xFFFFFFFFu;  // AND of the same
-    misc[2] = 0u;           // positive scores
-    misc[3] = 0xFFFFFFFFu;  // row minimum score word
+  // Keys of non-negative floats order like the values; the passes sort
+  // key - minimum over the bits where the keys can differ: from the lowest
+  // bit any key sets (all keys are multiples of it) to the top bit of the
+  // range.
+  const int npos = st.npos;
+  int lo = 0, hi = -1;
+  if (st.kmax > st.kmin) {
+    lo = __ffs(static_cast<int>(st.kor)) - 1;
+    hi = 31 - __clz(static_cast<int>(st.kmax - st.kmin));
   }
-  __syncthreads();
-    // Score words of non-negative floats order like the values; subtracting
-    // the row minimum keeps the order and leaves fewer bytes to sort.
-    uint32_t lo = 0xFFFFFFFFu, pos = 0u;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t w = sc0[i];
-      lo = min(lo, w);
-      pos += w != 0u;
-    }
-    lo = __reduce_min_sync(0xFFFFFFFFu, lo);
-    pos = __reduce_add_sync(0xFFFFFFFFu, pos);
-    if (lane == 0) {
-      atomicMin(&misc[3], lo);
-      atomicAdd(&misc[2], pos);
-    }
-    __syncthreads();
-    const uint32_t row_min = misc[3];
-    uint32_t o = 0u, a = 0xFFFFFFFFu;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t w = sc0[i] - row_min;
-      sc0[i] = w;
-      o |= w;
-      a &= w;
-    }
-    o = __reduce_or_sync(0xFFFFFFFFu, o);
-    a = __reduce_and_sync(0xFFFFFFFFu, a);
-    if (lane == 0) {
-      atomicOr(&misc[0], o);
-      atomicAnd(&misc[1], a);
-    }
-    __syncthreads();
-    const uint32_t vary = misc[0] ^ misc[1];
-    const int npos = static_cast<int>(misc[2]);
-    uint32_t* ks = sc0;
-    uint16_t* ps = nullptr;
-    stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, vary,
-                                                      reinterpret_cast<uint16_t*>(cnt), base);
+  uint32_t* ks = sc0;
+  uint16_t* ps = nullptr;
+  stable_sort32_by_score<kSortWarps, kSortMaxSlots>(&ks, &ps, sc1, ps1, ps0, n, st.kmin, lo, hi,
+                                                    reinterpret_cast<uint16_t*>(cnt), base);
     if (!zero_mode || npos >= m) {
       for (int i = threadIdx.x; i < top_k; i += blockDim.x)
         out[i] = i < m ? static_cast<int32_t>(ix[ps ? ps[i] : i]) : -1;
@@ -376,10 +398,20 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
+      stats_init(sm.misc);
       sm.misc[4] = 0u;           // largest exponent field of a positive accumulator
       sm.misc[5] = 0xFFFFFFFFu;  // lowest set bit (exponent of 2) over them, biased by 150
     }
-    merge_by_index(raw, n0, raw + n0, n1, sm.sc0, sm.ix);
+    __syncthreads();
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u, orr = 0u, pos = 0u, emax = 0u, pmin = 0xFFFFFFFFu;
+    merge_by_index(raw, n0, raw + n0, n1, sm.sc0, sm.ix, lo, hi, orr, pos, emax, pmin);
+    stats_reduce(lo, hi, orr, pos, sm.misc);
+    emax = __reduce_max_sync(0xFFFFFFFFu, emax);
+    pmin = __reduce_min_sync(0xFFFFFFFFu, pmin);
+    if (lane == 0) {
+      atomicMax(&sm.misc[4], emax);
+      atomicMin(&sm.misc[5], pmin);
+    }
     __syncthreads();
     // Ordering by relu(acc) is ordering by score = relu(fp32(acc) * scale), ties
     // included, when the scale is positive and no two distinct accumulators of
@@ -388,41 +420,31 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     // differ by 2 ulps of the larger score) and the smallest scores stay
     // normal.  Integer-valued index inputs give that.  Otherwise the keys
     // become the score words.
-    {
-      uint32_t emax = 0u, pmin = 0xFFFFFFFFu;
+    KeyStats st = stats_read(sm.misc);
+    const uint32_t em = sm.misc[4], pm = sm.misc[5];
+    // every positive accumulator is a multiple of 2^(pm - 150) >= 4 ulps of
+    // the largest (2^(em - 148)); the smallest score, >= 2^(pm - 150) * scale,
+    // is normal
+    const bool by_acc =
+        p.scale > 0.0f &&
+        (pm == 0xFFFFFFFFu ||
+         (pm >= em + 2u && __fmul_rn(ldexpf(1.0f, static_cast<int>(pm) - 150), p.scale) >= 1.17549435e-38f));
+    if (!by_acc) {
+      __syncthreads();  // everyone has read misc
+      if (threadIdx.x == 0) stats_init(sm.misc);
+      __syncthreads();
+      lo = 0xFFFFFFFFu, hi = 0u, orr = 0u, pos = 0u;
       for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t w = sm.sc0[i];
-        if (w) {
-          const uint32_t e = w >> 23;
-          const uint32_t mant = (w & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-          emax = max(emax, e);
-          pmin = min(pmin, e ? e + static_cast<uint32_t>(__ffs(static_cast<int>(mant)) - 1) : 0u);
-        }
+        const float sc = __fmul_rn(__uint_as_float(sm.sc0[i]), p.scale);
+        const uint32_t w = sc > 0.0f ? __float_as_uint(sc) : 0u;
+        sm.sc0[i] = w;
+        stats_add(w, lo, hi, orr, pos);
       }
-      emax = __reduce_max_sync(0xFFFFFFFFu, emax);
-      pmin = __reduce_min_sync(0xFFFFFFFFu, pmin);
-      if (lane == 0) {
-        atomicMax(&sm.misc[4], emax);
-        atomicMin(&sm.misc[5], pmin);
-      }
+      stats_reduce(lo, hi, orr, pos, sm.misc);
       __syncthreads();
-      const uint32_t em = sm.misc[4], pm = sm.misc[5];
-      // every positive accumulator is a multiple of 2^(pm - 150) >= 4 ulps of
-      // the largest (2^(em - 148)); the smallest score, >= 2^(pm - 150) * scale,
-      // is normal
-      const bool by_acc =
-          p.scale > 0.0f &&
-          (pm == 0xFFFFFFFFu ||
-           (pm >= em + 2u && __fmul_rn(ldexpf(1.0f, static_cast<int>(pm) - 150), p.scale) >= 1.17549435e-38f));
-      if (!by_acc) {
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-          const float sc = __fmul_rn(__uint_as_float(sm.sc0[i]), p.scale);
-          sm.sc0[i] = sc > 0.0f ? __float_as_uint(sc) : 0u;
-        }
-      }
-      __syncthreads();
+      st = stats_read(sm.misc);
     }
-    sort_emit(sm, n, m, zero_mode, t, p.top_k, p.indices + t * p.top_k);
+    sort_emit(sm, n, m, zero_mode, t, p.top_k, p.indices + t * p.top_k, st);
     __syncthreads();
   }
 }
@@ -604,6 +626,8 @@ __global__ void __launch_bounds__(kSortThreads, 1) fb_select_kernel(const FbPara
     // stable compaction of the keys in bins >= b, four consecutive keys per thread
     const unsigned long long* keys = p.scratch + static_cast<int64_t>(f) * p.L;
     uint32_t done = 0;
+    uint32_t slo = 0xFFFFFFFFu, shi = 0u, sor = 0u, spos = 0u;
+    if (threadIdx.x == 0) stats_init(misc);  // misc[0..3]; b and total are held in registers
     for (int s0 = 0; s0 < n; s0 += 4 * kSortThreads) {
       const int sb = s0 + 4 * threadIdx.x;
       unsigned long long k4[4];
@@ -629,15 +653,20 @@ __global__ void __launch_bounds__(kSortThreads, 1) fb_select_kernel(const FbPara
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         if (sb + q < n && static_cast<uint32_t>(k4[q] >> 51) >= b) {
-          sm.sc0[pos] = static_cast<uint32_t>(k4[q] >> 32);
+          const uint32_t w = static_cast<uint32_t>(k4[q] >> 32);
+          sm.sc0[pos] = w;
           sm.ix[pos] = static_cast<uint32_t>(sb + q);
+          stats_add(w, slo, shi, sor, spos);
           ++pos;
         }
       }
       done += all;
       __syncthreads();
     }
-    sort_emit(sm, static_cast<int>(total), m, false, t, p.top_k, p.indices + t * p.top_k);
+    stats_reduce(slo, shi, sor, spos, misc);
+    __syncthreads();
+    sort_emit(sm, static_cast<int>(total), m, false, t, p.top_k, p.indices + t * p.top_k,
+              stats_read(misc));
     __syncthreads();
   }
 }

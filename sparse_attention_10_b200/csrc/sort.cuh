@@ -106,7 +106,7 @@ __device__ unsigned long long* stable_sort_by_score(unsigned long long* a, unsig
 namespace dsa {
 
 // Stable pass on 32-bit keys with 16-bit payloads (positions):
-// (kout, pout) = (kin, pin) ordered by the `width`-bit digit (key >> shift),
+// (kout, pout) = (kin, pin) ordered by the `width`-bit digit ((key - kmin) >> shift),
 // width <= 9, DESCENDING, equal digits in input order.  pin == nullptr means
 // the identity payload.  Warp w owns items [w * chunk, (w + 1) * chunk), lane
 // order within each 32-item slot; ranks inside a warp come from
@@ -115,8 +115,8 @@ namespace dsa {
 // base [512].
 template <int WARPS, int SLOTS>
 __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint32_t* kout,
-                                 uint16_t* pout, int n, int shift, int width, uint16_t* cnt16,
-                                 uint32_t* base) {
+                                 uint16_t* pout, int n, uint32_t kmin, int shift, int width,
+                                 uint16_t* cnt16, uint32_t* base) {
   constexpr int kBins = 512;
   static_assert(WARPS * 32 >= kBins, "one thread per digit");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,7 +133,7 @@ __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint3
     if (j < slots) {
       const int i = warp * chunk + j * 32 + lane;
       const bool ok = i < n;
-      const uint32_t d = ok ? top - ((kin[i] >> shift) & top) : 512u;
+      const uint32_t d = ok ? top - (((kin[i] - kmin) >> shift) & top) : 512u;
       const uint32_t peers = __match_any_sync(0xFFFFFFFFu, d);
       const uint32_t before = ok ? wc[d] : 0u;
       dr[j] = (d << 16) | (before + __popc(peers & lt));
@@ -184,31 +184,29 @@ __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint3
   __syncthreads();
 }
 
-// Stable sort of (key, position) pairs, descending by key, over the bits that
-// differ among the keys (`vary` = OR ^ AND of the keys): the span from the
-// lowest to the highest differing bit is cut into equal digits of at most 9
-// bits, one pass each, least significant first.  Returns through *k / *p the
-// buffers holding the result; *p == nullptr means no pass ran (input order).
-// cnt16 needs WARPS * 512 16-bit counters, base 512 + WARPS words.
+// Stable sort of (key, position) pairs, descending by key, over bits lo..hi
+// of key - kmin (the bits where the keys can differ; hi < lo: all keys
+// equal): the span is cut into equal digits of at most 9 bits, one pass
+// each, least significant first.  Returns through *k / *p the buffers holding
+// the result; *p == nullptr means no pass ran (input order).  cnt16 needs
+// WARPS * 512 16-bit counters, base 512 + WARPS words.
 template <int WARPS, int SLOTS>
 __device__ void stable_sort32_by_score(uint32_t** k, uint16_t** p, uint32_t* k_alt,
-                                       uint16_t* p_alt, uint16_t* p_first, int n, uint32_t vary,
-                                       uint16_t* cnt16, uint32_t* base) {
+                                       uint16_t* p_alt, uint16_t* p_first, int n, uint32_t kmin,
+                                       int lo, int hi, uint16_t* cnt16, uint32_t* base) {
   uint32_t* kc = *k;
   uint16_t* pc = nullptr;             // identity until the first pass
   uint32_t* kn = k_alt;
   uint16_t* pn = p_first;
   uint16_t* spare = p_alt;
-  if (vary != 0u) {
-    const int lo = __ffs(static_cast<int>(vary)) - 1;
-    const int hi = 31 - __clz(static_cast<int>(vary));
+  if (hi >= lo) {
     const int span = hi - lo + 1;
     const int passes = (span + 8) / 9;
     const int width = (span + passes - 1) / passes;
     for (int q = 0; q < passes; ++q) {
       const int sh = lo + q * width;
       const int wd = min(width, hi + 1 - sh);
-      radix_pass32_var<WARPS, SLOTS>(kc, pc, kn, pn, n, sh, wd, cnt16, base);
+      radix_pass32_var<WARPS, SLOTS>(kc, pc, kn, pn, n, kmin, sh, wd, cnt16, base);
       uint32_t* tk = kc;
       kc = kn;
       kn = tk;
