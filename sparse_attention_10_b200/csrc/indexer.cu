@@ -37,8 +37,6 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kChunk = 16;        // columns per TMEM load in the epilogue
-constexpr int kStagePitch = 20;   // floats per thread in the epilogue staging area
-constexpr int kStagingBytes = kEpiWarps * 32 * kStagePitch * 4;
 constexpr int kMiscBytes = 1024;  // barriers, TMEM slot, abort flag
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kTileA = kBM * 32;   // bytes of one 32-byte K slice of the A tile
@@ -69,7 +67,7 @@ struct Params {
   int64_t Lq, Lk;
   int nkb, stages;
   Slices sl;
-  uint32_t off_b, off_stage, off_bar;
+  uint32_t off_b, off_bar;
   float scale;
   int mode;
   int n_items;
@@ -163,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + p.off_b;
-  float* staging = reinterpret_cast<float*>(smem + p.off_stage);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
   const int S = p.stages;
   // barrier slots
@@ -331,7 +328,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const int row_local = quarter * 32 + lane;
-    float* my_stage = staging + (ew * 32 + lane) * kStagePitch;
     uint32_t acc_it = 0;
     bool ok = true;
     for (int round = 0; ok; ++round) {
@@ -373,17 +369,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // turns the accumulator into relu(fp32(acc) * scale).
                 const int hits = __popc(pass);
                 if (count + hits <= p.cap) {
-                  uint32_t* st = reinterpret_cast<uint32_t*>(my_stage);
-                  uint4* st4 = reinterpret_cast<uint4*>(my_stage);
-#pragma unroll
-                  for (int q = 0; q < kChunk / 4; ++q)
-                    st4[q] = make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
                   uint2* dst = reinterpret_cast<uint2*>(my_cand + count);
                   const uint32_t nbase = 0xFFFFFFFFu - static_cast<uint32_t>(s0);
                   while (pass) {
                     const int q = __ffs(pass) - 1;
                     pass &= pass - 1;
-                    *dst++ = make_uint2(nbase - q, st[q]);
+                    // v[q] by a select tree over the 16 registers
+                    uint32_t t8[8], t4[4], t2[2];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) t8[e] = (q & 1) ? v[2 * e + 1] : v[2 * e];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) t4[e] = (q & 2) ? t8[2 * e + 1] : t8[2 * e];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) t2[e] = (q & 4) ? t4[2 * e + 1] : t4[2 * e];
+                    *dst++ = make_uint2(nbase - q, (q & 8) ? t2[1] : t2[0]);
                   }
                 }
                 count += hits;
@@ -602,7 +601,7 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   if (d_bytes % 32 != 0 || d_bytes <= 0 || a.d > DSA_MAX_INDEX_DIM) return DSA_ERR_UNSUPPORTED;
   const int nkb = d_bytes / 32;
   const uint32_t a_bytes = nkb * kTileA, stage_bytes = nkb * kTileB;
-  const int avail = kSmemLimit - 1024 - static_cast<int>(a_bytes) - kStagingBytes - kMiscBytes;
+  const int avail = kSmemLimit - 1024 - static_cast<int>(a_bytes) - kMiscBytes;
   const int stages = std::min(8, avail / static_cast<int>(stage_bytes));
   if (stages < 1) return DSA_ERR_UNSUPPORTED;
 
@@ -613,8 +612,7 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   p.nkb = nkb;
   p.stages = stages;
   p.off_b = a_bytes;
-  p.off_stage = a_bytes + stages * stage_bytes;
-  p.off_bar = p.off_stage + kStagingBytes;
+  p.off_bar = a_bytes + stages * stage_bytes;
   p.scale = a.scale;
   p.mode = a.mode;
   p.n_items = static_cast<int>((a.Lq + kBM - 1) / kBM);

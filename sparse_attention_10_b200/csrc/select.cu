@@ -424,11 +424,12 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     const uint32_t em = sm.misc[4], pm = sm.misc[5];
     // every positive accumulator is a multiple of 2^(pm - 150) >= 4 ulps of
     // the largest (2^(em - 148)); the smallest score, >= 2^(pm - 150) * scale,
-    // is normal
+    // is normal, and the largest score is finite (no ties at +inf)
     const bool by_acc =
         p.scale > 0.0f &&
         (pm == 0xFFFFFFFFu ||
-         (pm >= em + 2u && __fmul_rn(ldexpf(1.0f, static_cast<int>(pm) - 150), p.scale) >= 1.17549435e-38f));
+         (pm >= em + 2u && __fmul_rn(ldexpf(1.0f, static_cast<int>(pm) - 150), p.scale) >= 1.17549435e-38f &&
+          __fmul_rn(__uint_as_float(st.kmax), p.scale) < INFINITY));
     if (!by_acc) {
       __syncthreads();  // everyone has read misc
       if (threadIdx.x == 0) stats_init(sm.misc);
