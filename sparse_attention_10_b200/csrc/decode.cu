@@ -28,7 +28,7 @@ namespace dsa {
 namespace {
 
 constexpr int kScanThreads = 256;
-constexpr int kScanRowsPerCta = 4096;
+constexpr int kScanRowsPerCta = 2048;
 constexpr int kHistBins = 2048;           // score bits 30..20 (scores are >= +0)
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
@@ -372,15 +372,18 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   if (ncand <= kSmemKeys) {
     // Stable compaction of the candidates (score bin >= bin) in index order.
     uint32_t o_or = 0u, o_and = 0xFFFFFFFFu;
-    for (int s0 = 0; s0 < n; s0 += kSelThreads * 4) {
-      const int s = s0 + threadIdx.x * 4;
-      float v[4];
+    // eight consecutive scores per thread and round: the loads of a round
+    // are independent, so the rounds (each a block scan) are few
+    constexpr int kPer = 8;
+    for (int s0 = 0; s0 < n; s0 += kSelThreads * kPer) {
+      const int s = s0 + threadIdx.x * kPer;
+      float v[kPer];
       uint32_t flags = 0;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        v[k] = s + k < n ? sc[s + k] : 0.0f;
+      for (int k = 0; k < kPer; ++k) v[k] = s + k < n ? sc[s + k] : 0.0f;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k)
         if (s + k < n && (__float_as_uint(v[k]) >> 20) >= bin) flags |= 1u << k;
-      }
       const uint32_t c = __popc(flags);
       uint32_t incl = c;
 #pragma unroll
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
       __syncthreads();
       int pos = sh[2] + static_cast<int>(wsum[warp] + incl - c);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < kPer; ++k) {
         if (flags & (1u << k)) {
           const uint32_t bits = __float_as_uint(v[k]);
           o_or |= bits;
