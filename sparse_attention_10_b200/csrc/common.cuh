@@ -158,35 +158,8 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
       : "memory");
 }
 
-// 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (taddr.lane + i).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor (tcgen05 format, version 1) for a K-major
-// operand stored in 32-byte-swizzled atoms: rows of 32 bytes, 8-row groups
-// 256 bytes apart.  One descriptor covers one 32-byte slice of K.
-__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);       // start address
-  d |= static_cast<uint64_t>(1) << 16;                      // LBO (unused when K fits one atom)
-  d |= static_cast<uint64_t>(256 >> 4) << 32;               // SBO: 8 rows x 32 B
-  d |= static_cast<uint64_t>(1) << 46;                      // descriptor version (sm_100)
-  d |= static_cast<uint64_t>(6) << 61;                      // layout: 32-byte swizzle
-  return d;
 }
 
 // Shared-memory matrix descriptor for a K-major operand stored in swizzled
@@ -215,12 +188,6 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t M, uint
          | (fmt << 10)          // B format
          | ((N >> 3) << 17)     // N / 8
          | ((M >> 4) << 24);    // M / 16
-}
-
-// Monotone map of a float's bits to an unsigned key (larger float -> larger key).
-__device__ __forceinline__ uint32_t float_key(float f) {
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 }  // namespace dsa
