@@ -294,6 +294,19 @@ def test_prefill_full_workloads_sampled(dsa, name):
     assert stats["fallback_rows"] < w.L // 100, stats
 
 
+def test_prefill_128k_forced_fallback_rows(dsa, force_fallback):
+    # Full-size rows (up to 131072 keys each) through the grid-wide fallback:
+    # every 10007th row is forced there and compared with the oracle.
+    w = synth.WORKLOADS["prefill_128k"]
+    x = host_copy(synth.prefill_inputs_torch(w, device="cuda"))
+    force_fallback(10007)
+    idx, O, stats = run_prefill(dsa, x, w.top_k)
+    forced = np.arange(0, w.L, 10007, dtype=np.int64)
+    assert stats["fallback_rows"] >= len(forced), stats
+    check_index_properties(idx, w.top_k)
+    compare(x, w.idx_dtype, w.top_k, idx, O, rows=forced)
+
+
 # ------------------------------------------------------------------ decode
 
 def run_decode(dsa, xd, top_k):
