@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t r = r0 + u * RPL + rsub;
-      w[u] = r < c1 ? __ldg(reinterpret_cast<const uint4*>(rows + r * (LPR * 16) + sub * 16))
+      // streaming loads: the cache is read once and should not evict what
+      // the attention will gather
+      w[u] = r < c1 ? __ldcs(reinterpret_cast<const uint4*>(rows + r * (LPR * 16) + sub * 16))
                     : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
