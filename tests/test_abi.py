@@ -99,3 +99,10 @@ def test_python_binding_refuses_cpu_tensors(lib):
     q = torch.zeros((4, 128), dtype=torch.uint8)
     with pytest.raises(ValueError):
         dsa.dsa_indexer_scores(q, q)
+
+
+def test_force_fallback_hook_validates_and_resets(lib):
+    import sparse_attention_10_b200 as dsa
+    assert lib.dsa_debug_force_fallback(-1) == 1     # negative period rejected
+    dsa.dsa_debug_force_fallback(7)
+    dsa.dsa_debug_force_fallback(0)                  # back to normal
