@@ -116,6 +116,15 @@ def test_prefill_small_all_rows(dsa, L, top_k):
     compare(x, "fp8", top_k, idx, O)
 
 
+@pytest.mark.parametrize("L,top_k,H", [(1, 16, 16), (5, 16, 1), (129, 64, 16), (300, 300, 3), (777, 128, 16)])
+def test_prefill_small_head_dim_128(dsa, L, top_k, H):
+    # Head dim 128 runs the tcgen05 attention: single-key items, items shorter
+    # than one 128-key tile, fewer heads than the MMA's 16.
+    x = small_inputs(L, 128, H, 128, seed=17)
+    idx, O, _ = run_prefill(dsa, x, top_k)
+    compare(x, "fp8", top_k, idx, O)
+
+
 def test_prefill_d96_ragged(dsa):
     x = small_inputs(2333, 96, 16, 128, seed=5)
     idx, O, _ = run_prefill(dsa, x, 128)
