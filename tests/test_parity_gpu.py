@@ -360,6 +360,20 @@ def test_decode_index_formats(dsa, idx_dtype, d, top_k):
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
 
 
+@pytest.mark.parametrize("B", [75, 100, 200])
+def test_decode_batch_sizes(dsa, B):
+    """Batches that take 3, 2 and 2 key splits per sequence on 148 SMs; lengths 1..3000 leave
+    splits with no keys (a sequence shorter than its split count) and ragged last splits."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([1 + (i * 977) % 3000 for i in range(B)], dtype=np.int64)
+    lens[:3] = [1, 2, 3]
+    xd = synth.decode_inputs(w, lengths=lens)
+    idx, O = run_decode(dsa, xd, 512)
+    ri, ro = oracle.decode(xd, w.idx_dtype, 512)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
 def test_decode_full_workload(dsa):
     w = synth.WORKLOADS["decode_64x128k"]
     xd = host_copy(synth.decode_inputs_torch(w, device="cuda"))
