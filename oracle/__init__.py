@@ -149,3 +149,34 @@ def decode(inp: dict, idx_dtype: str, top_k: int, idx_scale=None, attn_scale=Non
                           d, D, _ptr(q_idx), _ptr(Q), H, top_k, idx_scale, attn_scale,
                           _ptr(indices), _ptr(O), nthreads)
     return indices, O
+
+
+def decode_paged(inp: dict, idx_dtype: str, top_k: int, idx_scale=None, attn_scale=None,
+                 want_o: bool = True, nthreads: int = 0):
+    """One decode step over a block-paged cache: indices [B, top_k] and O [B, H, D].
+
+    The DeepSeek Sparse Attention page (section 4.2) keeps the cache in token
+    blocks laid out on 128-byte boundaries.  Read here as: row s of sequence b
+    lives in block ``block_table[b, s // block_size]`` at offset
+    ``s % block_size`` of pools shaped [num_blocks, block_size, ...].  The
+    oracle reads each sequence's rows out in order and takes the ordinary
+    decode step on them; indices are positions within the sequence.
+    """
+    table = np.asarray(inp["block_table"])
+    lens = np.asarray(inp["seq_lens"], dtype=np.int64)
+    bs = inp["k_idx_blocks"].shape[1]
+    rows = []
+    for b in range(lens.shape[0]):
+        s = np.arange(int(lens[b]))
+        rows.append(table[b, s // bs].astype(np.int64) * bs + s % bs)
+    rows = np.concatenate(rows)
+    seq_start = np.zeros(lens.shape[0] + 1, dtype=np.int64)
+    seq_start[1:] = np.cumsum(lens)
+    flat = {"k_idx": inp["k_idx_blocks"].reshape(-1, inp["k_idx_blocks"].shape[2])[rows],
+            "q_idx": inp["q_idx"], "seq_start": seq_start}
+    if want_o:
+        D = inp["K_blocks"].shape[2]
+        flat["K"] = inp["K_blocks"].reshape(-1, D)[rows]
+        flat["V"] = inp["V_blocks"].reshape(-1, D)[rows]
+        flat["Q"] = inp["Q"]
+    return decode(flat, idx_dtype, top_k, idx_scale, attn_scale, want_o, nthreads)

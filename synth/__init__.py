@@ -34,6 +34,7 @@ __all__ = [
     "GOLDEN", "SEED", "mix64", "draws", "uniform_ints", "fp8_bytes_of_ints",
     "bf16_bits_of_ints", "bf16_bits_of_f32", "normal_bf16", "Workload",
     "WORKLOADS", "prefill_inputs", "decode_inputs", "decode_lengths", "stream_key",
+    "paged_layout", "paged_decode_inputs", "paged_decode_inputs_torch",
 ]
 
 GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -176,6 +177,7 @@ WORKLOADS = {
 
 # tensor ids inside a workload's streams
 _T_QIDX, _T_KIDX, _T_Q, _T_K, _T_V, _T_BOOST, _T_LEN = 1, 2, 3, 4, 5, 6, 7
+_T_PAGE, _T_PAD_KIDX, _T_PAD_K, _T_PAD_V = 8, 9, 10, 11
 
 
 def _encode_ints(v: np.ndarray, idx_dtype: str) -> np.ndarray:
@@ -263,6 +265,78 @@ def decode_inputs(w: Workload, seed: int = SEED, lengths: Optional[np.ndarray] =
         out["K"] = _prefix_normal(seed, w.cid, _T_K, total * w.D).reshape(total, w.D)
         out["V"] = _prefix_normal(seed, w.cid, _T_V, total * w.D).reshape(total, w.D)
     return out
+
+
+def paged_layout(lengths, block_size: int, seed: int = SEED, spare_blocks: int = 3):
+    """Placement of a decode batch in a block-paged cache.
+
+    Sequence b occupies ceil(len_b / block_size) blocks of ``block_size`` rows.
+    Those blocks, plus ``spare_blocks`` that no sequence uses, are shuffled by a
+    seeded permutation (the order of splitmix64 draws), so neighbouring blocks
+    of one sequence land at unrelated places in the pool.  Row s of sequence b
+    is pool row ``block_table[b, s // block_size] * block_size + s % block_size``.
+
+    Returns ``block_table`` [B, max_blocks] int32 (-1 past each sequence's last
+    block) and ``src`` [num_blocks * block_size] int64: for every pool row, the
+    row of the contiguous cache (sequences back to back, as decode_inputs lays
+    them out) that it holds, or -1 for rows no sequence reaches.
+    """
+    lengths = np.asarray(lengths, dtype=np.int64)
+    assert block_size >= 1 and (block_size & (block_size - 1)) == 0
+    nblk = (lengths + block_size - 1) // block_size
+    used = int(nblk.sum())
+    n_total = used + spare_blocks
+    order = np.argsort(draws(stream_key(seed, n_total, block_size, _T_PAGE), 0, n_total), kind="stable")
+    B = lengths.shape[0]
+    table = np.full((B, max(1, int(nblk.max()))), -1, dtype=np.int32)
+    src = np.full(n_total * block_size, -1, dtype=np.int64)
+    nxt, first = 0, 0
+    for b in range(B):
+        for j in range(int(nblk[b])):
+            phys = int(order[nxt])
+            nxt += 1
+            table[b, j] = phys
+            n = min(block_size, int(lengths[b]) - j * block_size)
+            src[phys * block_size: phys * block_size + n] = first + j * block_size + np.arange(n)
+        first += int(lengths[b])
+    return table, src
+
+
+def _fill_pool(rows: np.ndarray, src: np.ndarray, pad: np.ndarray) -> np.ndarray:
+    out = pad.copy()
+    m = src >= 0
+    out[m] = rows[src[m]]
+    return out
+
+
+def paged_decode_inputs(w: Workload, lengths, block_size: int, seed: int = SEED,
+                        spare_blocks: int = 3) -> dict:
+    """decode_inputs placed in a block-paged cache (paged_layout).
+
+    The rows are those of decode_inputs(w, seed, lengths); pool rows that no
+    sequence reaches hold draws of their own streams, so a read of a wrong row
+    changes scores and outputs.  Returns k_idx_blocks [num_blocks, block_size,
+    d_idx], K_blocks / V_blocks [num_blocks, block_size, D], block_table,
+    seq_lens [B] int32, q_idx, Q, lengths, B, block_size, and the contiguous
+    inputs under "contiguous".
+    """
+    xd = decode_inputs(w, seed, lengths=lengths)
+    table, src = paged_layout(xd["lengths"], block_size, seed, spare_blocks)
+    nrows = src.shape[0]
+    nb = nrows // block_size
+    pad_i = _encode_ints(uniform_ints(stream_key(seed, w.cid, _T_PAD_KIDX), nrows * w.d_idx)
+                         .reshape(nrows, w.d_idx), w.idx_dtype)
+    pad_k = _prefix_normal(seed, w.cid, _T_PAD_K, nrows * w.D).reshape(nrows, w.D)
+    pad_v = _prefix_normal(seed, w.cid, _T_PAD_V, nrows * w.D).reshape(nrows, w.D)
+    return {
+        "k_idx_blocks": _fill_pool(xd["k_idx"], src, pad_i).reshape(nb, block_size, w.d_idx),
+        "K_blocks": _fill_pool(xd["K"], src, pad_k).reshape(nb, block_size, w.D),
+        "V_blocks": _fill_pool(xd["V"], src, pad_v).reshape(nb, block_size, w.D),
+        "block_table": table,
+        "seq_lens": xd["lengths"].astype(np.int32),
+        "q_idx": xd["q_idx"], "Q": xd["Q"], "lengths": xd["lengths"], "B": xd["B"],
+        "block_size": block_size, "contiguous": xd,
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -365,4 +439,27 @@ def decode_inputs_torch(w: Workload, seed: int = SEED, device="cuda") -> dict:
         "Q": normal_bf16_torch(stream_key(seed, w.cid, _T_Q), B * w.H * w.D, device).view(B, w.H, w.D),
         "K": normal_bf16_torch(stream_key(seed, w.cid, _T_K), total * w.D, device).view(total, w.D),
         "V": normal_bf16_torch(stream_key(seed, w.cid, _T_V), total * w.D, device).view(total, w.D),
+    }
+
+
+def paged_decode_inputs_torch(xd: dict, block_size: int, seed: int = SEED, spare_blocks: int = 3) -> dict:
+    """A device copy of a decode batch (decode_inputs_torch) placed in a block-paged
+    cache by paged_layout; rows no sequence reaches are zero."""
+    import torch
+    table, src = paged_layout(xd["lengths"], block_size, seed, spare_blocks)
+    dev = xd["k_idx"].device
+    s = torch.from_numpy(src).to(dev)
+    m = s >= 0
+
+    def pool(x):
+        out = x.new_zeros((s.numel(),) + tuple(x.shape[1:]))
+        out[m] = x[s[m]]
+        return out.view((s.numel() // block_size, block_size) + tuple(x.shape[1:]))
+
+    return {
+        "k_idx_blocks": pool(xd["k_idx"]), "K_blocks": pool(xd["K"]), "V_blocks": pool(xd["V"]),
+        "block_table": torch.from_numpy(table).to(dev),
+        "seq_lens": torch.from_numpy(np.asarray(xd["lengths"], dtype=np.int32)).to(dev),
+        "q_idx": xd["q_idx"], "Q": xd["Q"], "lengths": xd["lengths"], "B": xd["B"],
+        "block_size": block_size,
     }

@@ -320,3 +320,65 @@ def test_decode_is_last_row_of_each_sequence(oracle_mod):
             oracle_mod.default_index_scale(w.d_idx))
         sc = np.where(sc > 0, sc, np.float32(0))
         assert idx[b].tolist() == stable_topk(sc, k).tolist()
+
+
+# ---------------------------------------------------------------- paged decode
+
+def test_paged_decode_literal_layout(oracle_mod):
+    """A block-paged cache written out by hand (block size 2): the paged step equals
+    the step over the same rows stored back to back."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    flat = synth.decode_inputs(w, lengths=np.array([3, 5], dtype=np.int64))
+    # sequence 0 (rows 0..2 of the flat cache) in blocks 4, 1;
+    # sequence 1 (rows 3..7) in blocks 0, 5, 2; block 3 is unused
+    table = np.array([[4, 1, -1], [0, 5, 2]], dtype=np.int32)
+    holds = [3, 4, 2, None, 7, None, None, None, 0, 1, 5, 6]   # pool row -> flat row
+    rng = np.random.default_rng(5)
+
+    def pool(x):
+        out = rng.integers(0, 1 << (8 * x.itemsize), size=(12,) + x.shape[1:]).astype(x.dtype)
+        for r, f in enumerate(holds):
+            if f is not None:
+                out[r] = x[f]
+        return out.reshape((6, 2) + x.shape[1:])
+
+    paged = {"k_idx_blocks": pool(flat["k_idx"]), "K_blocks": pool(flat["K"]),
+             "V_blocks": pool(flat["V"]), "block_table": table,
+             "seq_lens": np.array([3, 5], dtype=np.int32), "q_idx": flat["q_idx"], "Q": flat["Q"]}
+    for k in (1, 4, 16):
+        pi, po = oracle_mod.decode_paged(paged, "fp8", k)
+        ri, ro = oracle_mod.decode(flat, "fp8", k)
+        assert np.array_equal(pi, ri) and np.array_equal(po, ro)
+    # a wrong block (sequence 1's middle block pointed at the unused one) changes the result
+    bad = dict(paged, block_table=np.array([[4, 1, -1], [0, 3, 2]], dtype=np.int32))
+    bi, bo = oracle_mod.decode_paged(bad, "fp8", 4)
+    ri, ro = oracle_mod.decode(flat, "fp8", 4)
+    assert not (np.array_equal(bi, ri) and np.array_equal(bo, ro))
+
+
+@pytest.mark.parametrize("block_size", [1, 4, 64])
+def test_paged_layout_places_every_row_once(block_size):
+    lengths = np.array([1, 63, 64, 65, 200], dtype=np.int64)
+    table, src = synth.paged_layout(lengths, block_size, spare_blocks=2)
+    starts = np.concatenate([[0], np.cumsum(lengths)])
+    placed = src[src >= 0]
+    assert np.array_equal(np.sort(placed), np.arange(int(lengths.sum())))
+    for b, n in enumerate(lengths):
+        s = np.arange(int(n))
+        assert np.array_equal(src[table[b, s // block_size].astype(np.int64) * block_size + s % block_size],
+                              starts[b] + s)
+        used = -(-int(n) // block_size)
+        assert (table[b, used:] == -1).all()
+    nb = src.shape[0] // block_size
+    assert nb == int((-(-lengths // block_size)).sum()) + 2
+    assert sorted(table[table >= 0].tolist()) == sorted(set(table[table >= 0].tolist()))
+
+
+def test_paged_decode_inputs_match_contiguous(oracle_mod):
+    w = synth.WORKLOADS["decode_64x128k"]
+    lengths = np.array([1, 2, 100, 2049, 300], dtype=np.int64)
+    for bs in (1, 16, 4096):
+        xp = synth.paged_decode_inputs(w, lengths, bs)
+        pi, po = oracle_mod.decode_paged(xp, "fp8", 256)
+        ri, ro = oracle_mod.decode(xp["contiguous"], "fp8", 256)
+        assert np.array_equal(pi, ri) and np.array_equal(po, ro)
