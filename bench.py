@@ -496,6 +496,39 @@ def main():
         if dsa.dsa_sync_status(stream) != 0:
             raise RuntimeError("device-side error in decode")
 
+        # the same batch in a block-paged cache: blocks of 64 rows placed by a seeded permutation
+        bsz = 64
+        xp = synth.paged_decode_inputs_torch(xd, bsz, seed=seed)
+        wsp = torch.empty(dsa.dsa_decode_paged_workspace_size(wd.B, int(lengths.max()), wd.d_idx, 0, wd.H,
+                                                               wd.D, wd.top_k), dtype=torch.uint8, device=dev)
+        Op, idp = torch.empty_like(Od), torch.empty_like(idd)
+
+        def pstep():
+            dsa.dsa_decode_paged(xp["k_idx_blocks"], xp["K_blocks"], xp["V_blocks"], xp["block_table"],
+                                 xp["seq_lens"], xp["q_idx"], xp["Q"], wd.top_k, int(lengths.max()), O=Op,
+                                 indices=idp, workspace=wsp, stream=stream)
+
+        for _ in range(args.warmup):
+            pstep()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(nd):
+            pstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        pms = max_over_ranks(e0.elapsed_time(e1))
+        if dsa.dsa_sync_status(stream) != 0:
+            raise RuntimeError("device-side error in paged decode")
+        decode["paged"] = {
+            "value": world * wd.B * nd / (pms / 1000.0), "unit": "tok/s", "ms_per_step": pms / nd,
+            "layout": f"k_idx/K/V pools of {xp['k_idx_blocks'].shape[0]} blocks x {bsz} rows, "
+                      f"block table [{wd.B}, {xp['block_table'].shape[1]}] int32, seeded block order",
+            "matches_contiguous": bool(torch.equal(idp, idd) and torch.equal(Op, Od))}
+        del xp, wsp
+
     # --- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -142,6 +142,43 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
                       float attn_scale, void* O, int32_t* indices, void* workspace,
                       size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace dsa_decode_paged needs (planned for B * max_len rows). */
+size_t dsa_decode_paged_workspace_size(int B, int64_t max_len, int d_idx, int idx_dtype, int H,
+                                       int D, int top_k);
+
+/*
+ * dsa_decode_paged — dsa_decode over a block-paged cache.  The DeepSeek
+ * Sparse Attention page (section 4.2) keeps the cache in token blocks laid
+ * out on 128-byte boundaries; read here as pools of fixed-size blocks and a
+ * per-sequence block table, so a sequence grows by appending a block and
+ * blocks need not be contiguous or in order (several sequences may share
+ * one).  Row s of sequence b (0 <= s < seq_lens[b]) is row
+ * s % block_size of block block_table[b * max_blocks + s / block_size].
+ *   k_idx        device [num_blocks, block_size, d_idx] FP8 E4M3 or BF16
+ *   K, V         device [num_blocks, block_size, D] BF16
+ *   block_table  device [B, max_blocks] int32; entries past a sequence's
+ *                last block are not read
+ *   seq_lens     device [B] int32, each in [1, max_len] and at most
+ *                max_blocks * block_size
+ *   block_size   a power of two in [1, 65536];
+ *                num_blocks * block_size <= 2^31 - 1
+ *   max_len      host bound on every seq_lens[b] (sizes the scan grid and
+ *                the workspace: dsa_decode_paged_workspace_size)
+ * Every other argument, output and limit is that of dsa_decode; indices are
+ * positions within the sequence (0 .. len_b - 1), not pool rows.  The
+ * device checks the lengths and every block id a sequence reaches
+ * (0 <= id < num_blocks) before any kernel reads through the table; a
+ * failure makes the call a no-op that records DSA_ERR_INVALID_ARG in the
+ * status word (dsa_sync_status).  Host-side argument errors return
+ * DSA_ERR_INVALID_ARG at once and enqueue nothing.
+ */
+dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int64_t num_blocks,
+                            int block_size, const int32_t* block_table, int max_blocks,
+                            const int32_t* seq_lens, int B, int64_t max_len, int idx_dtype,
+                            int d_idx, int D, const void* q_idx, const void* Q, int H, int top_k,
+                            float idx_scale, float attn_scale, void* O, int32_t* indices,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * dsa_sync_status — synchronise `stream`, then read and clear the current
  * device's status word (the first device-side error since the last read).

@@ -19,6 +19,7 @@ __all__ = [
     "dsa_prefill_workspace_size", "dsa_prefill", "dsa_decode_workspace_size", "dsa_decode",
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "dsa_debug_force_fallback", "IDX_FP8_E4M3", "IDX_BF16",
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
+    "dsa_decode_paged_workspace_size", "dsa_decode_paged",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -58,6 +59,9 @@ def load() -> ctypes.CDLL:
         "dsa_debug_wait_timeout": ([ctypes.c_uint64, P], I),
         "dsa_debug_force_fallback": ([I], I),
         "dsa_decode_static": ([P, P, P, P, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P], I),
+        "dsa_decode_paged_workspace_size": ([I, I64, I, I, I, I, I], SZ),
+        "dsa_decode_paged": ([P, P, P, I64, I, P, I, P, I, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ,
+                              P], I),
         "dsa_stage_timing": ([I], I),
         "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
     }
@@ -185,6 +189,49 @@ def dsa_decode(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_start:
                         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                         _stream(stream))
     _check(st, "dsa_decode")
+    return O, indices
+
+
+def dsa_decode_paged_workspace_size(B: int, max_len: int, d_idx: int, idx_dtype: int, H: int, D: int,
+                                    top_k: int) -> int:
+    return int(load().dsa_decode_paged_workspace_size(B, max_len, d_idx, idx_dtype, H, D, top_k))
+
+
+def dsa_decode_paged(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block_table: torch.Tensor,
+                     seq_lens: torch.Tensor, q_idx: torch.Tensor, Q: torch.Tensor, top_k: int, max_len: int,
+                     idx_scale: Optional[float] = None, attn_scale: Optional[float] = None,
+                     O: Optional[torch.Tensor] = None, indices: Optional[torch.Tensor] = None,
+                     want_indices: bool = True, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """One decode step over a block-paged cache -> (O [B, H, D] bf16, indices [B, top_k] or None).
+
+    k_idx [num_blocks, block_size, d_idx], K/V [num_blocks, block_size, D],
+    block_table [B, max_blocks] int32, seq_lens [B] int32 (all on the device)."""
+    lib = load()
+    B, d = q_idx.shape
+    _, H, D = Q.shape
+    num_blocks, block_size = k_idx.shape[0], k_idx.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if block_table.dim() != 2 or block_table.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_table must be [B, max_blocks] and seq_lens [B]")
+    idt = _idx_dtype(q_idx)
+    dev = q_idx.device
+    if O is None:
+        O = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    if indices is None and want_indices:
+        indices = torch.empty((B, top_k), dtype=torch.int32, device=dev)
+    if workspace is None:
+        need = dsa_decode_paged_workspace_size(B, int(max_len), d, idt, H, D, top_k)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = lib.dsa_decode_paged(_dev(k_idx, "k_idx"), _dev(K, "K"), _dev(V, "V"), num_blocks, block_size,
+                              _dev(block_table, "block_table"), block_table.shape[1],
+                              _dev(seq_lens, "seq_lens"), B, int(max_len), idt, d, D, _dev(q_idx, "q_idx"),
+                              _dev(Q, "Q"), H, top_k, _scale(idx_scale), _scale(attn_scale), _dev(O, "O"),
+                              _dev(indices, "indices") if indices is not None else None,
+                              _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(st, "dsa_decode_paged")
     return O, indices
 
 

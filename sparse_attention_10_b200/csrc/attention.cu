@@ -86,6 +86,8 @@ struct AttnParams {
   __nv_bfloat16* O;
   float* part;
   const int* invalid;
+  const int32_t* block_table;   // paged decode cache, else null
+  int bt_ld, bs_log2;
 };
 
 template <int D>
@@ -141,8 +143,10 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     // rows a query may read: its causal prefix (prefill) or its sequence (decode)
     const int row_limit = p.seq_start ? static_cast<int>(p.seq_start[q + 1] - row_base)
                                       : static_cast<int>(min64(q + 1, 0x7FFFFFFF));
-    const __nv_bfloat16* Kb = p.K + row_base * D;
-    const __nv_bfloat16* Vb = p.V + row_base * D;
+    // a paged cache's key rows are absolute (translated below)
+    const int64_t kv_base = p.block_table ? 0 : row_base;
+    const __nv_bfloat16* Kb = p.K + kv_base * D;
+    const __nv_bfloat16* Vb = p.V + kv_base * D;
 
     // Q rows (heads >= H are zero) and this item's key list, clamped.
     // (asynchronous copies: every row of Q and the whole key list in flight at once)
@@ -158,7 +162,11 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     __syncthreads();
     for (int i = tid; i < n; i += kAttnThreads) {
       const int s = sIds[i];
-      sIds[i] = (s >= 0 && s < row_limit) ? s : -1;
+      int r = (s >= 0 && s < row_limit) ? s : -1;
+      if (p.block_table && r >= 0)   // position in the sequence -> row of the block pool
+        r = (__ldg(p.block_table + q * p.bt_ld + (r >> p.bs_log2)) << p.bs_log2) |
+            (r & ((1 << p.bs_log2) - 1));
+      sIds[i] = r;
     }
     __syncthreads();
 
@@ -382,8 +390,9 @@ dsa_status launch_combine(const AttnLaunch& a, cudaStream_t stream) {
 
 template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
-  AttnParams p{a.Q, a.K, a.V, a.idx, a.ld_idx, a.nq, a.H, a.scale_log2, a.top_k, a.seq_start,
-               a.nsplit, a.O, a.part, a.invalid};
+  AttnParams p{a.Q,      a.K,    a.V,       a.idx,         a.ld_idx, a.nq,
+               a.H,      a.scale_log2, a.top_k, a.seq_start, a.nsplit, a.O,
+               a.part,   a.invalid, a.block_table, a.bt_ld, a.bs_log2};
   const size_t smem = AttnSmem<D>::kBytes;
   static_assert(AttnSmem<D>::kStages * 2 * AttnSmem<D>::kTile >=
                     (4 * 16 * 2 + 4 * 16 * AttnSmem<D>::kMergeRow) * 4,
@@ -403,10 +412,10 @@ dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream) {
-  // Split launches (decode: 8 splits of 256 keys per query) are short items,
-  // where the mma.sync kernel's lower per-item latency wins (0.030 vs 0.039 ms
-  // for 64 x 2048 keys).
-  if (a.nsplit == 1 && attention_tc_supported(a)) {
+  // Split launches (decode: 2-8 splits per query) are short items, where the
+  // mma.sync kernel's lower per-item latency wins (0.030 vs 0.039 ms for
+  // 64 x 2048 keys in 256-key items).  Paged caches take the mma.sync kernel.
+  if (a.nsplit == 1 && !a.block_table && attention_tc_supported(a)) {
     const dsa_status st = launch_attention_tc(a, stream);
     return st != DSA_OK ? st : launch_combine<128>(a, stream);
   }

@@ -100,6 +100,44 @@ __global__ void validate_kernel(const int64_t* seq_start, int B, int64_t total_r
   }
 }
 
+// Paged cache: every length in [1, max_len] and within its block-table row,
+// every block a sequence reaches in [0, num_blocks).  CTA b also writes the
+// sum of the lengths before sequence b (and, for the last, the total), which
+// the later stages use as seq_start.
+__global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t max_len,
+                                      const int32_t* table, int bt_ld, int bs_log2,
+                                      int64_t num_blocks, int64_t* seq_start_out, int* invalid) {
+  __shared__ long long wsum[32];
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  long long before = 0;
+  for (int i = threadIdx.x; i < b; i += blockDim.x) before += seq_lens[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xFFFFFFFFu, before, o);
+  if (lane == 0) wsum[warp] = before;
+  const int64_t len = seq_lens[b];
+  bool bad = len < 1 || len > max_len || ((len - 1) >> bs_log2) >= bt_ld;
+  if (!bad) {
+    const int64_t nblk = ((len - 1) >> bs_log2) + 1;
+    const int32_t* row = table + static_cast<int64_t>(b) * bt_ld;
+    for (int64_t j = threadIdx.x; j < nblk; j += blockDim.x) {
+      const int32_t v = row[j];
+      bad |= v < 0 || v >= num_blocks;
+    }
+  }
+  const int any_bad = __syncthreads_or(bad);
+  if (threadIdx.x == 0) {
+    long long start = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) start += wsum[w];
+    seq_start_out[b] = start;
+    if (b == B - 1) seq_start_out[B] = start + len;
+    if (any_bad) {
+      *invalid = 1;
+      record_error(DSA_ERR_INVALID_ARG);
+    }
+  }
+}
+
 struct ScanParams {
   const void* k_idx;
   const void* q_idx;
@@ -109,9 +147,17 @@ struct ScanParams {
   float* scores;
   unsigned int* hist;
   const int* invalid;
+  const int32_t* block_table;   // paged cache (PAGED kernels only)
+  int bt_ld, bs_log2;
 };
 
-template <int ESIZE>
+// Cache row of row s of sequence b in a paged cache.
+__device__ __forceinline__ int64_t paged_row(const ScanParams& p, int b, int64_t s) {
+  const int32_t blk = __ldg(p.block_table + static_cast<int64_t>(b) * p.bt_ld + (s >> p.bs_log2));
+  return (static_cast<int64_t>(blk) << p.bs_log2) | (s & ((int64_t(1) << p.bs_log2) - 1));
+}
+
+template <int ESIZE, bool PAGED>
 __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanParams p) {
   __shared__ float qf[DSA_MAX_INDEX_DIM];
   __shared__ unsigned int hist[kHistBins];
@@ -138,7 +184,8 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
     const int64_t s = s0 + threadIdx.x;
     uint32_t bin = 0;
     if (s < c1) {
-      float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, base + s, p.d), p.scale);
+      const int64_t row = PAGED ? paged_row(p, b, s) : base + s;
+      float sc = __fmul_rn(dot_row<ESIZE>(qf, p.k_idx, row, p.d), p.scale);
       sc = sc > 0.0f ? sc : 0.0f;
       p.scores[base + s] = sc;
       bin = __float_as_uint(sc) >> 20;
@@ -155,12 +202,17 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
 // lanes share a row, each holding its 16-byte slice of the query in
 // registers; a warp load covers 32 / LPR consecutive rows, eight loads are in
 // flight per lane, and log2(LPR) shuffles finish each row's dot product.
-template <int ESIZE, int LPR>
+//
+// PAGED: the cache is block-paged; the CTA's slice of its sequence's block
+// table (at most kScanRowsPerCta entries, block sizes being powers of two) is
+// staged in shared memory, and each row address is looked up there.
+template <int ESIZE, int LPR, bool PAGED>
 __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const ScanParams p) {
   constexpr int RPL = 32 / LPR;                 // rows per warp load
   constexpr int U = 8;                          // loads in flight per lane
   constexpr int VALS = 16 / ESIZE;              // index values per 16-byte slice
   __shared__ unsigned int hist[kHistBins];
+  __shared__ int32_t blk[PAGED ? kScanRowsPerCta : 1];
   if (*p.invalid) return;
   const int b = blockIdx.y;
   const int64_t base = p.seq_start[b];
@@ -182,16 +234,28 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
     }
   }
   for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  const int64_t j0 = PAGED ? c0 >> p.bs_log2 : 0;
+  const int64_t off_mask = (int64_t(1) << p.bs_log2) - 1;
+  if (PAGED) {
+    const int64_t j1 = (c1 - 1) >> p.bs_log2;
+    const int32_t* trow = p.block_table + static_cast<int64_t>(b) * p.bt_ld;
+    for (int64_t j = j0 + threadIdx.x; j <= j1; j += blockDim.x) blk[j - j0] = trow[j];
+  }
   __syncthreads();
-  const uint8_t* rows = static_cast<const uint8_t*>(p.k_idx) + base * (LPR * 16);
+  const uint8_t* rows = static_cast<const uint8_t*>(p.k_idx) + (PAGED ? 0 : base * (LPR * 16));
   for (int64_t r0 = c0 + warp * RPL * U; r0 < c1; r0 += (kScanThreads / 32) * RPL * U) {
     uint4 w[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t r = r0 + u * RPL + rsub;
+      int64_t cr = r;   // cache row
+      if (PAGED) {
+        const int64_t rr = r < c1 ? r : c0;
+        cr = (static_cast<int64_t>(blk[(rr >> p.bs_log2) - j0]) << p.bs_log2) | (rr & off_mask);
+      }
       // streaming loads: the cache is read once and should not evict what
       // the attention will gather
-      w[u] = r < c1 ? __ldcs(reinterpret_cast<const uint4*>(rows + r * (LPR * 16) + sub * 16))
+      w[u] = r < c1 ? __ldcs(reinterpret_cast<const uint4*>(rows + cr * (LPR * 16) + sub * 16))
                     : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
@@ -472,30 +536,44 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
     out[i] = i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
 }
 
+template <bool PAGED>
+void launch_scan(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
+  if (esize == 1 && lpr == 8)
+    decode_scan_rows_kernel<1, 8, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (esize == 1 && lpr == 4)
+    decode_scan_rows_kernel<1, 4, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (esize == 1 && lpr == 16)
+    decode_scan_rows_kernel<1, 16, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (esize == 2 && lpr == 8)
+    decode_scan_rows_kernel<2, 8, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (esize == 2 && lpr == 16)
+    decode_scan_rows_kernel<2, 16, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else if (esize == 1)
+    decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+  else
+    decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+}
+
 }  // namespace
 
 dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
   if (cudaMemsetAsync(a.hist, 0, sizeof(unsigned int) * kHistBins * a.B, stream) != cudaSuccess)
     return DSA_ERR_CUDA;
-  validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.invalid);
-  ScanParams sp{a.k_idx, a.q_idx, a.d, a.seq_start, a.scale, a.scores, a.hist, a.invalid};
+  if (a.seq_lens)
+    validate_paged_kernel<<<a.B, 256, 0, stream>>>(a.seq_lens, a.B, a.max_len, a.block_table,
+                                                   a.bt_ld, a.bs_log2, a.num_blocks,
+                                                   a.seq_start_out, a.invalid);
+  else
+    validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.invalid);
+  ScanParams sp{a.k_idx,   a.q_idx,   a.d,           a.seq_start, a.scale, a.scores,
+                a.hist,    a.invalid, a.block_table, a.bt_ld,     a.bs_log2};
   const dim3 grid(static_cast<unsigned int>((a.max_len + kScanRowsPerCta - 1) / kScanRowsPerCta),
                   static_cast<unsigned int>(a.B));
   const int lpr = a.d * a.esize / 16;  // 16-byte slices per index row
-  if (a.esize == 1 && lpr == 8)
-    decode_scan_rows_kernel<1, 8><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (a.esize == 1 && lpr == 4)
-    decode_scan_rows_kernel<1, 4><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (a.esize == 1 && lpr == 16)
-    decode_scan_rows_kernel<1, 16><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (a.esize == 2 && lpr == 8)
-    decode_scan_rows_kernel<2, 8><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (a.esize == 2 && lpr == 16)
-    decode_scan_rows_kernel<2, 16><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (a.esize == 1)
-    decode_scan_kernel<1><<<grid, kScanThreads, 0, stream>>>(sp);
+  if (a.seq_lens)
+    launch_scan<true>(sp, grid, a.esize, lpr, stream);
   else
-    decode_scan_kernel<2><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_scan<false>(sp, grid, a.esize, lpr, stream);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
 
   DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid};

@@ -107,10 +107,11 @@ static int decode_splits(int B) {
 }
 
 struct DecodePlan {
-  size_t off_counters, off_scores, off_hist, off_keys, off_indices, off_part, total;
+  size_t off_counters, off_scores, off_hist, off_keys, off_indices, off_part, off_seq, total;
 };
 
-DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k) {
+// paged: one more array, the running sum of the lengths [B + 1] (int64)
+DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k, bool paged = false) {
   DecodePlan p{};
   size_t o = 0;
   p.off_counters = o;
@@ -125,6 +126,10 @@ DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k) {
   o = align_up(o + static_cast<size_t>(B) * top_k * sizeof(int32_t));
   p.off_part = o;
   o = align_up(o + static_cast<size_t>(B) * kDecodeSplits * H * (D + 2) * sizeof(float));
+  if (paged) {
+    p.off_seq = o;
+    o = align_up(o + static_cast<size_t>(B + 1) * sizeof(int64_t));
+  }
   p.total = o;
   return p;
 }
@@ -187,6 +192,110 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
   if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, limit_ns, nullptr);  // nothing arrives
   __syncthreads();
   if (threadIdx.x == 0) mbar_arrive(smem_u32(&bar));  // leave the barrier complete
+}
+
+constexpr int64_t kMaxDecodeLen = (int64_t(1) << 31) - 1;
+constexpr int kMaxBlockSize = 1 << 16;
+
+// One decode call: a contiguous cache (seq_start) or a paged one (seq_lens,
+// block_table); the entry points check what is particular to each.
+struct DecodeCall {
+  const void* k_idx;
+  const void* K;
+  const void* V;
+  const int64_t* seq_start;      // contiguous cache, else null
+  const int32_t* seq_lens;       // paged cache, else null
+  const int32_t* block_table;
+  int bt_ld, bs_log2;
+  int64_t num_blocks;
+  int B;
+  int64_t total_rows;            // rows the workspace is planned for
+  int64_t max_len;
+  int idx_dtype, d_idx, D;
+  const void* q_idx;
+  const void* Q;
+  int H, top_k;
+  float idx_scale, attn_scale;
+  void* O;
+  int32_t* indices;
+  void* workspace;
+  size_t workspace_bytes;
+  cudaStream_t stream;
+};
+
+dsa_status run_decode(const DecodeCall& c) {
+  const bool paged = c.seq_lens != nullptr;
+  if (!c.k_idx || !c.K || !c.V || !c.q_idx || !c.Q || !c.O || !c.workspace)
+    return DSA_ERR_INVALID_ARG;
+  for (const void* ptr : {c.k_idx, c.K, c.V, c.q_idx, c.Q, static_cast<const void*>(c.O)})
+    if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
+  if (c.indices && !aligned16(c.indices)) return DSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(c.workspace) & 255) != 0) return DSA_ERR_INVALID_ARG;
+  if (c.B < 1 || c.max_len < 1 || c.max_len > kMaxDecodeLen) return DSA_ERR_INVALID_ARG;
+  if (c.top_k < 1 || c.top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
+  if (c.H < 1 || c.H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
+  if (c.D != 64 && c.D != 128) return DSA_ERR_UNSUPPORTED;
+  dsa_status st = check_index_dims(c.idx_dtype, c.d_idx);
+  if (st != DSA_OK) return st;
+  const DecodePlan plan = plan_decode(c.B, c.total_rows, c.H, c.D, c.top_k, paged);
+  if (c.workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t s = c.stream;
+  uint8_t* ws = static_cast<uint8_t*>(c.workspace);
+  int32_t* idx = c.indices ? c.indices : reinterpret_cast<int32_t*>(ws + plan.off_indices);
+  if (cudaMemsetAsync(ws + plan.off_counters, 0, 64 * sizeof(int), s) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  int64_t* seq_ws = paged ? reinterpret_cast<int64_t*>(ws + plan.off_seq) : nullptr;
+  const int64_t* seq_start = paged ? seq_ws : c.seq_start;
+
+  DecodeLaunch dl{};
+  dl.k_idx = c.k_idx;
+  dl.q_idx = c.q_idx;
+  dl.esize = esize_of(c.idx_dtype);
+  dl.d = c.d_idx;
+  dl.seq_start = seq_start;
+  dl.B = c.B;
+  dl.total_rows = c.total_rows;
+  dl.max_len = c.max_len;
+  dl.scale = default_scale(c.idx_scale, c.d_idx);
+  dl.top_k = c.top_k;
+  dl.scores = reinterpret_cast<float*>(ws + plan.off_scores);
+  dl.hist = reinterpret_cast<unsigned int*>(ws + plan.off_hist);
+  dl.indices = idx;
+  dl.keys = reinterpret_cast<unsigned long long*>(ws + plan.off_keys);
+  dl.invalid = reinterpret_cast<int*>(ws + plan.off_counters) + 8;
+  dl.seq_lens = c.seq_lens;
+  dl.block_table = c.block_table;
+  dl.bt_ld = c.bt_ld;
+  dl.bs_log2 = c.bs_log2;
+  dl.num_blocks = c.num_blocks;
+  dl.seq_start_out = seq_ws;
+  {
+    StageScope scope(5, 3, s);  // validate + scan + select (timed together)
+    if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
+  }
+
+  AttnLaunch at{};
+  at.Q = static_cast<const __nv_bfloat16*>(c.Q);
+  at.K = static_cast<const __nv_bfloat16*>(c.K);
+  at.V = static_cast<const __nv_bfloat16*>(c.V);
+  at.kv_rows = paged ? c.num_blocks << c.bs_log2 : c.total_rows;
+  at.idx = idx;
+  at.ld_idx = c.top_k;
+  at.nq = c.B;
+  at.H = c.H;
+  at.D = c.D;
+  at.scale_log2 = default_scale(c.attn_scale, c.D) * 1.4426950408889634f;
+  at.top_k = c.top_k;
+  at.seq_start = seq_start;
+  at.nsplit = decode_splits(c.B);
+  at.O = static_cast<__nv_bfloat16*>(c.O);
+  at.part = reinterpret_cast<float*>(ws + plan.off_part);
+  at.invalid = dl.invalid;
+  at.block_table = c.block_table;
+  at.bt_ld = c.bt_ld;
+  at.bs_log2 = c.bs_log2;
+  StageScope scope(7, 2, s);
+  return launch_attention(at, s);
 }
 
 }  // namespace
@@ -373,69 +482,83 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
                       const void* q_idx, const void* Q, int H, int top_k, float idx_scale,
                       float attn_scale, void* O, int32_t* indices, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  if (!k_idx || !K || !V || !seq_start || !q_idx || !Q || !O || !workspace)
+  if (!seq_start || (reinterpret_cast<uintptr_t>(seq_start) & 7) != 0 || total_rows < 1)
     return DSA_ERR_INVALID_ARG;
-  for (const void* ptr : {k_idx, K, V, q_idx, Q, static_cast<const void*>(O)})
-    if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
-  if (indices && !aligned16(indices)) return DSA_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
-      (reinterpret_cast<uintptr_t>(seq_start) & 7) != 0)
-    return DSA_ERR_INVALID_ARG;
-  if (B < 1 || total_rows < 1 || max_len < 1 || max_len > (int64_t(1) << 31) - 1)
-    return DSA_ERR_INVALID_ARG;
-  if (top_k < 1 || top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
-  if (H < 1 || H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
-  dsa_status st = check_index_dims(idx_dtype, d_idx);
-  if (st != DSA_OK) return st;
-  const DecodePlan plan = plan_decode(B, total_rows, H, D, top_k);
-  if (workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  int32_t* idx = indices ? indices : reinterpret_cast<int32_t*>(ws + plan.off_indices);
-  if (cudaMemsetAsync(ws + plan.off_counters, 0, 64 * sizeof(int), s) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  DecodeCall c{};
+  c.k_idx = k_idx;
+  c.K = K;
+  c.V = V;
+  c.seq_start = seq_start;
+  c.B = B;
+  c.total_rows = total_rows;
+  c.max_len = max_len;
+  c.idx_dtype = idx_dtype;
+  c.d_idx = d_idx;
+  c.D = D;
+  c.q_idx = q_idx;
+  c.Q = Q;
+  c.H = H;
+  c.top_k = top_k;
+  c.idx_scale = idx_scale;
+  c.attn_scale = attn_scale;
+  c.O = O;
+  c.indices = indices;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  c.stream = static_cast<cudaStream_t>(stream);
+  return run_decode(c);
+}
 
-  DecodeLaunch dl{};
-  dl.k_idx = k_idx;
-  dl.q_idx = q_idx;
-  dl.esize = esize_of(idx_dtype);
-  dl.d = d_idx;
-  dl.seq_start = seq_start;
-  dl.B = B;
-  dl.total_rows = total_rows;
-  dl.max_len = max_len;
-  dl.scale = default_scale(idx_scale, d_idx);
-  dl.top_k = top_k;
-  dl.scores = reinterpret_cast<float*>(ws + plan.off_scores);
-  dl.hist = reinterpret_cast<unsigned int*>(ws + plan.off_hist);
-  dl.indices = idx;
-  dl.keys = reinterpret_cast<unsigned long long*>(ws + plan.off_keys);
-  dl.invalid = reinterpret_cast<int*>(ws + plan.off_counters) + 8;
-  {
-    StageScope scope(5, 3, s);  // validate + scan + select (timed together)
-    if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
-  }
+size_t dsa_decode_paged_workspace_size(int B, int64_t max_len, int d_idx, int idx_dtype, int H,
+                                       int D, int top_k) {
+  (void)d_idx; (void)idx_dtype;
+  if (B < 1 || max_len < 1 || max_len > kMaxDecodeLen || H < 1 || top_k < 1) return 0;
+  return plan_decode(B, static_cast<int64_t>(B) * max_len, H, D, top_k, true).total;
+}
 
-  AttnLaunch at{};
-  at.Q = static_cast<const __nv_bfloat16*>(Q);
-  at.K = static_cast<const __nv_bfloat16*>(K);
-  at.V = static_cast<const __nv_bfloat16*>(V);
-  at.kv_rows = total_rows;
-  at.idx = idx;
-  at.ld_idx = top_k;
-  at.nq = B;
-  at.H = H;
-  at.D = D;
-  at.scale_log2 = default_scale(attn_scale, D) * 1.4426950408889634f;
-  at.top_k = top_k;
-  at.seq_start = seq_start;
-  at.nsplit = decode_splits(B);
-  at.O = static_cast<__nv_bfloat16*>(O);
-  at.part = reinterpret_cast<float*>(ws + plan.off_part);
-  at.invalid = dl.invalid;
-  StageScope scope(7, 2, s);
-  return launch_attention(at, s);
+dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int64_t num_blocks,
+                            int block_size, const int32_t* block_table, int max_blocks,
+                            const int32_t* seq_lens, int B, int64_t max_len, int idx_dtype,
+                            int d_idx, int D, const void* q_idx, const void* Q, int H, int top_k,
+                            float idx_scale, float attn_scale, void* O, int32_t* indices,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (!block_table || !seq_lens || (reinterpret_cast<uintptr_t>(block_table) & 3) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (block_size < 1 || block_size > kMaxBlockSize || (block_size & (block_size - 1)) != 0)
+    return DSA_ERR_INVALID_ARG;
+  if (num_blocks < 1 || num_blocks > INT32_MAX / block_size || max_blocks < 1 || B < 1 ||
+      max_len < 1 || max_len > kMaxDecodeLen)
+    return DSA_ERR_INVALID_ARG;
+  DecodeCall c{};
+  c.k_idx = k_idx;
+  c.K = K;
+  c.V = V;
+  c.seq_lens = seq_lens;
+  c.block_table = block_table;
+  c.bt_ld = max_blocks;
+  int lg = 0;
+  while ((1 << lg) < block_size) ++lg;
+  c.bs_log2 = lg;
+  c.num_blocks = num_blocks;
+  c.B = B;
+  c.total_rows = static_cast<int64_t>(B) * max_len;
+  c.max_len = max_len;
+  c.idx_dtype = idx_dtype;
+  c.d_idx = d_idx;
+  c.D = D;
+  c.q_idx = q_idx;
+  c.Q = Q;
+  c.H = H;
+  c.top_k = top_k;
+  c.idx_scale = idx_scale;
+  c.attn_scale = attn_scale;
+  c.O = O;
+  c.indices = indices;
+  c.workspace = workspace;
+  c.workspace_bytes = workspace_bytes;
+  c.stream = static_cast<cudaStream_t>(stream);
+  return run_decode(c);
 }
 
 dsa_status dsa_sync_status(void* stream) {

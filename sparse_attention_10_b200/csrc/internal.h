@@ -92,6 +92,10 @@ struct AttnLaunch {
   __nv_bfloat16* O;            // [nq, H, D] (nsplit == 1)
   float* part;                 // [nq, nsplit, H, D + 2] (nsplit > 1)
   const int* invalid;          // nonzero: skip all work (decode inputs failed validation)
+  // paged decode cache (null: K/V rows of query q start at seq_start[q]): key s of query q
+  // is row (block_table[q * bt_ld + (s >> bs_log2)] << bs_log2) | (s & (2^bs_log2 - 1))
+  const int32_t* block_table;
+  int bt_ld, bs_log2;
 };
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream);
@@ -113,10 +117,19 @@ struct DecodeLaunch {
   float scale;
   int top_k;
   float* scores;               // [total_rows]
-  unsigned int* hist;          // [B, 4096]
+  unsigned int* hist;          // [B, 2048]
   int32_t* indices;            // [B, top_k]
   unsigned long long* keys;    // [total_rows] scratch (many-candidate rows)
-  int* invalid;                // set when seq_start fails validation
+  int* invalid;                // set when seq_start (or the paged inputs) fail validation
+  // Paged cache (seq_lens non-null): row s of sequence b is k_idx row
+  // (block_table[b * bt_ld + (s >> bs_log2)] << bs_log2) | (s & (2^bs_log2 - 1)).
+  // The validator writes the running sum of the lengths into seq_start_out (then
+  // seq_start == seq_start_out), so scores and scratch stay indexed by sequence.
+  const int32_t* seq_lens;
+  const int32_t* block_table;
+  int bt_ld, bs_log2;
+  int64_t num_blocks;
+  int64_t* seq_start_out;
 };
 
 dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream);

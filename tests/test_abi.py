@@ -86,6 +86,30 @@ def test_decode_rejects_bad_arguments(lib):
     assert dec(ws_bytes=10) == 3
 
 
+def test_decode_paged_rejects_bad_arguments(lib):
+    def dec(bt=16, lens=16, nb=100, bs=64, mb=8, B=2, max_len=500, top_k=64, H=16, D=128, d=128,
+            kidx=16, ws_bytes=1 << 40):
+        return lib.dsa_decode_paged(P(kidx), P(16), P(16), nb, bs, P(bt), mb, P(lens), B, max_len, 0, d,
+                                    D, P(16), P(16), H, top_k, float("nan"), float("nan"), P(16), None,
+                                    P(256), ws_bytes, None)
+    assert dec(bt=0) == 1 and dec(lens=0) == 1        # null
+    assert dec(bt=18) == 1 and dec(lens=6) == 1       # int32 arrays must be 4-byte aligned
+    assert dec(kidx=8) == 1                           # pools 16-byte aligned
+    assert dec(bs=0) == 1 and dec(bs=48) == 1 and dec(bs=1 << 17) == 1   # power of two <= 65536
+    assert dec(nb=0) == 1
+    assert dec(nb=1 << 26, bs=64) == 1                # pool rows beyond 2^31 - 1
+    assert dec(mb=0) == 1
+    assert dec(B=0) == 1 and dec(max_len=0) == 1 and dec(max_len=1 << 31) == 1
+    assert dec(top_k=4096) == 1 and dec(H=0) == 1
+    assert dec(D=80) == 2
+    assert dec(ws_bytes=10) == 3
+    need = lib.dsa_decode_paged_workspace_size(2, 500, 128, 0, 16, 128, 64)
+    assert need > lib.dsa_decode_workspace_size(2, 1000, 128, 0, 16, 128, 64)   # + the length sums
+    assert dec(ws_bytes=need - 1) == 3
+    assert lib.dsa_decode_paged_workspace_size(0, 500, 128, 0, 16, 128, 64) == 0
+    assert lib.dsa_decode_paged_workspace_size(2, 0, 128, 0, 16, 128, 64) == 0
+
+
 def test_indexer_scores_rejects_bad_arguments(lib):
     f = lib.dsa_indexer_scores
     assert f(None, P(16), 0, 128, float("nan"), 4, 4, P(16), None) == 1

@@ -383,6 +383,94 @@ def test_decode_full_workload(dsa):
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
 
 
+# ------------------------------------------------------------------ paged decode
+
+def run_decode_paged(dsa, xp, top_k, max_len=None):
+    t = {k: to_dev(xp[k]) for k in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens",
+                                    "q_idx", "Q")}
+    O, idx = dsa.dsa_decode_paged(t["k_idx_blocks"], t["K_blocks"].view(torch.bfloat16),
+                                  t["V_blocks"].view(torch.bfloat16), t["block_table"], t["seq_lens"],
+                                  t["q_idx"], t["Q"].view(torch.bfloat16), top_k,
+                                  int(xp["lengths"].max()) if max_len is None else max_len)
+    return idx, O
+
+
+@pytest.mark.parametrize("block_size,idx_dtype,d,D,top_k", [
+    (1, "fp8", 128, 128, 256),       # one row per block
+    (16, "fp8", 128, 128, 2048),
+    (64, "bf16", 160, 128, 512),     # rows of 320 bytes: the generic scan kernel
+    (2048, "bf16", 128, 128, 128),   # one block per scan chunk
+    (4096, "fp8", 64, 64, 300),      # blocks longer than a scan chunk; head dim 64
+])
+def test_decode_paged_matches_oracle(dsa, block_size, idx_dtype, d, D, top_k):
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["decode_64x128k"], d_idx=d, idx_dtype=idx_dtype, D=D)
+    lens = np.array([1, 2, 100, 2047, 2048, 2049, 4097, 9000, 20001], dtype=np.int64)
+    xp = synth.paged_decode_inputs(w, lens, block_size)
+    idx, O = run_decode_paged(dsa, xp, top_k)
+    assert dsa.dsa_sync_status() == 0
+    ri, ro = oracle.decode_paged(xp, idx_dtype, top_k)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    got = O.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_decode_paged_shared_blocks(dsa):
+    """Two sequences whose block tables point at the same blocks (a shared
+    prefix) read the same rows: equal inputs give equal results."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([3000, 5000], dtype=np.int64)
+    xp = synth.paged_decode_inputs(w, lens, 64)
+    table = xp["block_table"].copy()
+    n0 = -(-3000 // 64)
+    table[1, :n0] = table[0, :n0]          # sequence 1 starts with sequence 0's blocks
+    shared = dict(xp, block_table=table)
+    idx, O = run_decode_paged(dsa, shared, 2048)
+    assert dsa.dsa_sync_status() == 0
+    ri, ro = oracle.decode_paged(shared, "fp8", 2048)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    got = O.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_decode_paged_rejects_bad_table_on_device(dsa):
+    """A block id outside the pool, or a length past max_len, is caught by the
+    device-side check before any kernel reads through the table: the call
+    records DSA_ERR_INVALID_ARG and the next valid call is unaffected."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([100, 700, 50], dtype=np.int64)
+    xp = synth.paged_decode_inputs(w, lens, 64)
+    nb = xp["k_idx_blocks"].shape[0]
+    bad = xp["block_table"].copy()
+    bad[1, 5] = nb                          # sequence 1 reaches block 5 (rows 320..383)
+    run_decode_paged(dsa, dict(xp, block_table=bad), 256)
+    assert dsa.dsa_sync_status() == 1
+    run_decode_paged(dsa, xp, 256, max_len=600)   # sequence 1 is longer than max_len
+    assert dsa.dsa_sync_status() == 1
+    idx, O = run_decode_paged(dsa, xp, 256)
+    assert dsa.dsa_sync_status() == 0
+    ri, _ = oracle.decode_paged(xp, "fp8", 256, want_o=False)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+
+
+def test_decode_paged_full_workload(dsa):
+    """The 64-sequence decode batch (65K-131K cached rows each) in blocks of 64
+    rows placed by a seeded permutation."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    xd = synth.decode_inputs_torch(w, device="cuda")
+    xp = synth.paged_decode_inputs_torch(xd, 64)
+    O, idx = dsa.dsa_decode_paged(xp["k_idx_blocks"], xp["K_blocks"].view(torch.bfloat16),
+                                  xp["V_blocks"].view(torch.bfloat16), xp["block_table"], xp["seq_lens"],
+                                  xp["q_idx"], xp["Q"].view(torch.bfloat16), w.top_k,
+                                  int(xp["lengths"].max()))
+    assert dsa.dsa_sync_status() == 0
+    idx, O = idx.cpu().numpy(), O.view(torch.int16).cpu().numpy().view(np.uint16)
+    del xp
+    ri, ro = oracle.decode(host_copy(xd), w.idx_dtype, w.top_k)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
 def test_device_generator_matches_numpy_definition():
     k = synth.stream_key(5, 6)
     a = synth.normal_bf16(k, 3_000_001)
