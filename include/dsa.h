@@ -134,7 +134,7 @@ size_t dsa_decode_workspace_size(int B, int64_t total_rows, int d_idx, int idx_d
  *   indices    device [B, top_k] int32, written when non-null (rank order,
  *              -1 padded), positions relative to the sequence's first row
  *   max_len    host bound on every len_b (sizes the scan grid)
- * Limits as dsa_prefill; max_len <= 2^31 - 1.
+ * Limits as dsa_prefill; 1 <= B <= 65535, max_len <= 2^31 - 1.
  */
 dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int64_t* seq_start,
                       int B, int64_t total_rows, int64_t max_len, int idx_dtype, int d_idx, int D,

@@ -195,6 +195,7 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
 }
 
 constexpr int64_t kMaxDecodeLen = (int64_t(1) << 31) - 1;
+constexpr int kMaxDecodeBatch = 65535;  // sequences are the scan grid's y extent
 constexpr int kMaxBlockSize = 1 << 16;
 
 // One decode call: a contiguous cache (seq_start) or a paged one (seq_lens,
@@ -231,7 +232,8 @@ dsa_status run_decode(const DecodeCall& c) {
     if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
   if (c.indices && !aligned16(c.indices)) return DSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(c.workspace) & 255) != 0) return DSA_ERR_INVALID_ARG;
-  if (c.B < 1 || c.max_len < 1 || c.max_len > kMaxDecodeLen) return DSA_ERR_INVALID_ARG;
+  if (c.B < 1 || c.B > kMaxDecodeBatch || c.max_len < 1 || c.max_len > kMaxDecodeLen)
+    return DSA_ERR_INVALID_ARG;
   if (c.top_k < 1 || c.top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
   if (c.H < 1 || c.H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
   if (c.D != 64 && c.D != 128) return DSA_ERR_UNSUPPORTED;

@@ -80,6 +80,7 @@ def test_decode_rejects_bad_arguments(lib):
     assert dec(seq=0) == 1
     assert dec(seq=20) == 1        # int64 array must be 8-byte aligned
     assert dec(B=0) == 1
+    assert dec(B=65536, total=1 << 20) == 1   # sequences are a grid dimension
     assert dec(max_len=0) == 1
     assert dec(top_k=4096) == 1
     assert dec(D=80) == 2
@@ -99,7 +100,8 @@ def test_decode_paged_rejects_bad_arguments(lib):
     assert dec(nb=0) == 1
     assert dec(nb=1 << 26, bs=64) == 1                # pool rows beyond 2^31 - 1
     assert dec(mb=0) == 1
-    assert dec(B=0) == 1 and dec(max_len=0) == 1 and dec(max_len=1 << 31) == 1
+    assert dec(B=0) == 1 and dec(B=65536) == 1
+    assert dec(max_len=0) == 1 and dec(max_len=1 << 31) == 1
     assert dec(top_k=4096) == 1 and dec(H=0) == 1
     assert dec(D=80) == 2
     assert dec(ws_bytes=10) == 3

@@ -55,3 +55,28 @@ def test_decode_lengths_in_range():
     w = synth.WORKLOADS["decode_64x128k"]
     n = synth.decode_lengths(w)
     assert n.shape == (64,) and n.min() >= 65536 and n.max() <= 131072
+
+
+def test_paged_inputs_torch_match_numpy():
+    """The device-side builder of a paged cache (used by the benchmark) places the
+    rows exactly as the numpy one the parity tests use."""
+    import torch
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([5, 130, 64, 1], dtype=np.int64)
+    xp = synth.paged_decode_inputs(w, lens, 16)
+    xd = xp["contiguous"]
+    xt = {"k_idx": torch.from_numpy(xd["k_idx"]), "K": torch.from_numpy(xd["K"].view(np.int16)),
+          "V": torch.from_numpy(xd["V"].view(np.int16)), "q_idx": torch.from_numpy(xd["q_idx"]),
+          "Q": torch.from_numpy(xd["Q"].view(np.int16)), "lengths": lens, "B": 4}
+    pt = synth.paged_decode_inputs_torch(xt, 16)
+    assert np.array_equal(pt["block_table"].numpy(), xp["block_table"])
+    assert np.array_equal(pt["seq_lens"].numpy(), xp["seq_lens"])
+    table = xp["block_table"]
+    for name, ref in (("k_idx_blocks", xp["k_idx_blocks"]), ("K_blocks", xp["K_blocks"].view(np.int16)),
+                      ("V_blocks", xp["V_blocks"].view(np.int16))):
+        got = pt[name].numpy()
+        assert got.shape == ref.shape
+        for b, n in enumerate(lens):     # every row a sequence reaches is the same
+            s = np.arange(int(n))
+            blk, off = table[b, s // 16], s % 16
+            assert np.array_equal(got[blk, off], ref[blk, off])
