@@ -382,3 +382,47 @@ def test_paged_decode_inputs_match_contiguous(oracle_mod):
         pi, po = oracle_mod.decode_paged(xp, "fp8", 256)
         ri, ro = oracle_mod.decode(xp["contiguous"], "fp8", 256)
         assert np.array_equal(pi, ri) and np.array_equal(po, ro)
+
+
+# ---------------------------------------------------------------- scale overrides
+
+def _fp8_of_ints(v):
+    return torch.from_numpy(np.asarray(v, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def _bf16_times2(bits):
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16) * 2
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_scale_overrides_are_applied(oracle_mod):
+    """Doubling an operand (exact in FP8 and BF16) and halving its scale leaves every
+    result unchanged bit for bit, while the default scale on the doubled operand does not:
+    so a supplied idx_scale / attn_scale is used, not replaced by the default."""
+    L, d, H, D, k = 48, 64, 2, 32, 8
+    key = synth.stream_key(11, 48, 64)
+    qi = synth.uniform_ints(key, L * d).reshape(L, d)
+    ki = synth.uniform_ints(key, L * d, start=L * d).reshape(L, d)
+    x = {"q_idx": _fp8_of_ints(qi), "k_idx": _fp8_of_ints(ki),
+         "Q": synth.normal_bf16(synth.stream_key(11, 1), L * H * D).reshape(L, H, D),
+         "K": synth.normal_bf16(synth.stream_key(11, 2), L * D).reshape(L, D),
+         "V": synth.normal_bf16(synth.stream_key(11, 3), L * D).reshape(L, D)}
+    s_idx, s_att = oracle_mod.default_index_scale(d), 1.0 / np.sqrt(D)
+    q2 = _fp8_of_ints(2 * qi)
+    a = oracle_mod.indexer_scores(x["q_idx"], x["k_idx"], "fp8")
+    assert np.array_equal(oracle_mod.indexer_scores(q2, x["k_idx"], "fp8", scale=s_idx / 2), a)
+    assert np.array_equal(oracle_mod.indexer_scores(q2, x["k_idx"], "fp8"), 2 * a) and a.max() > 0
+
+    x2 = dict(x, Q=_bf16_times2(x["Q"]))
+    ri, ro = oracle_mod.prefill_rows(x, "fp8", k)
+    si, so = oracle_mod.prefill_rows(x2, "fp8", k, attn_scale=s_att / 2)
+    assert np.array_equal(si, ri) and np.array_equal(so, ro)
+    _, to = oracle_mod.prefill_rows(x2, "fp8", k)
+    assert not np.array_equal(to, ro)
+
+    lens = np.array([1, 7, 40], dtype=np.int64)
+    xd = synth.decode_inputs(synth.WORKLOADS["decode_64x128k"], lengths=lens)
+    xd2 = dict(xd, Q=_bf16_times2(xd["Q"]))
+    di, do = oracle_mod.decode(xd, "fp8", k)
+    ei, eo = oracle_mod.decode(xd2, "fp8", k, attn_scale=1.0 / np.sqrt(xd["Q"].shape[2]) / 2)
+    assert np.array_equal(ei, di) and np.array_equal(eo, do)
