@@ -8,8 +8,10 @@ indexer with fused filter + exact select + gathered attention.  `value` is
 whole-job prefill queries/s (each rank runs its own sequence: weak scaling,
 no data-path collective).  The decode rows of the path (64 sequences with
 cached lengths in [65536, 131072], top_k 2048) are timed in their own K-step
-loop and reported under "decode".  Inputs are synthetic and seeded; each
-step's working set (~9 GB) is far larger than the 126 MB L2.
+loop and reported under "decode", and again from a block-paged copy of the
+same cache (dsa_decode_paged, 64-row blocks) under "decode.paged".  Inputs
+are synthetic and seeded; each step's working set (~9 GB) is far larger than
+the 126 MB L2.
 
 --impl reference times the CPU oracle (the plain restatement the tests check
 against) on a bounded sample of query rows per step, on the host's cores.
