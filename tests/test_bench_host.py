@@ -1,5 +1,6 @@
 """Host-side pieces of bench.py: the max-over-ranks reduction across two gloo
-ranks on CPU (the N > 1 timing path), work accounting and the profile lookup."""
+ranks on CPU (the N > 1 timing path), work accounting, the profile lookup and
+the reference arm (the CPU oracle) with its JSON line."""
 import os
 import socket
 import sys
@@ -57,3 +58,34 @@ def test_profiled_traffic_requires_matching_source(tmp_path, monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
     assert bench.profiled_traffic("no_such_kernel", "prefill_128k", "bench.py") is None
+
+
+def _bench(args, env_extra):
+    import json
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py")] + args, cwd=ROOT, env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    return [json.loads(ln) for ln in lines]
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` times the oracle on the host and prints one JSON
+    line with the contract's keys (no GPU needed)."""
+    (line,) = _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "0", "WORLD_SIZE": "1"})
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["steps"] == 1
+    assert line["config"]["workload"].startswith("prefill_128k")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"] and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    assert _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
