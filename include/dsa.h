@@ -11,7 +11,8 @@
  *                keys, then ordinary softmax attention runs over those keys;
  *   section 4.1  precision: FP8 index stage, BF16 attention stage;
  *   section 4.2  memory: all query heads share one K/V (MQA); rows are laid
- *                out on 128-byte boundaries;
+ *                out on 128-byte boundaries, the cache in token blocks
+ *                (dsa_decode_paged);
  *   section 7.2  per-length settings (FP8 at 32K/64K, BF16 index at 128K).
  * Readings where the page is silent (stated once here, used everywhere):
  *   - causal: query t sees keys s <= t, the diagonal included;
@@ -32,8 +33,9 @@
  *     distinct workspaces may run concurrently.
  *   - Argument errors are reported synchronously by the return value and
  *     nothing is enqueued.  Errors found on the device (a bounded wait that
- *     ran out) are recorded in a per-device status word that
- *     dsa_sync_status() reads and clears.
+ *     ran out; decode lengths or block ids that fail the device-side checks)
+ *     are recorded in a per-device status word that dsa_sync_status() reads
+ *     and clears.
  *   - idx_scale / attn_scale: pass NaN to use index_dim^-0.5 / D^-0.5
  *     (each rounded to float32).
  */
