@@ -243,15 +243,28 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   }
   __syncthreads();
   const uint8_t* rows = static_cast<const uint8_t*>(p.k_idx) + (PAGED ? 0 : base * (LPR * 16));
+  // A warp step covers RPL * U rows starting at a multiple of RPL * U; when a
+  // block holds at least that many rows they all lie in one block, so one
+  // lookup per step serves every load.
+  constexpr int kStepLog2 = LPR == 4 ? 6 : LPR == 8 ? 5 : 4;   // log2(RPL * U)
+  static_assert((1 << kStepLog2) == RPL * U, "rows per warp step");
+  const bool one_block = PAGED && p.bs_log2 >= kStepLog2;
   for (int64_t r0 = c0 + warp * RPL * U; r0 < c1; r0 += (kScanThreads / 32) * RPL * U) {
     uint4 w[U];
+    int64_t step_cr = 0;   // cache row of r0 (one-block steps)
+    if (one_block)
+      step_cr = (static_cast<int64_t>(blk[(r0 >> p.bs_log2) - j0]) << p.bs_log2) | (r0 & off_mask);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int64_t r = r0 + u * RPL + rsub;
       int64_t cr = r;   // cache row
       if (PAGED) {
-        const int64_t rr = r < c1 ? r : c0;
-        cr = (static_cast<int64_t>(blk[(rr >> p.bs_log2) - j0]) << p.bs_log2) | (rr & off_mask);
+        if (one_block) {
+          cr = step_cr + (u * RPL + rsub);
+        } else {
+          const int64_t rr = r < c1 ? r : c0;
+          cr = (static_cast<int64_t>(blk[(rr >> p.bs_log2) - j0]) << p.bs_log2) | (rr & off_mask);
+        }
       }
       // streaming loads: the cache is read once and should not evict what
       // the attention will gather
