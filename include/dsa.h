@@ -255,6 +255,12 @@ dsa_status dsa_debug_force_fallback(int period);
  * leaves its contents behind (each call clears what it needs zeroed), so
  * calls whose work overlaps on the GPU — on different streams, or from
  * different threads — race and corrupt each other: serialise them.
+ *
+ * The block belongs to the device that is current when the call is made:
+ * `stream` must be a stream of that device's primary context, and O must be
+ * device memory of that device (checked: DSA_ERR_INVALID_ARG otherwise).
+ * There is no workspace to hand to dsa_last_stats, so its counters are not
+ * available for calls made through this entry point.
  */
 #define DSA_DECODE_STATIC_SCRATCH_BYTES (18u << 20)
 dsa_status dsa_decode_static(const void* k_idx, const void* K, const void* V,

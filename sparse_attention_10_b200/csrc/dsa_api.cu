@@ -655,6 +655,16 @@ extern "C" dsa_status dsa_decode_static(const void* k_idx, const void* K, const 
   if (need > DSA_DECODE_STATIC_SCRATCH_BYTES) return DSA_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DSA_ERR_CUDA;
+  // The block's address is only valid on the device it was looked up for: the
+  // output must live on the current device.
+  if (O) {
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, O) != cudaSuccess) {
+      cudaGetLastError();
+      return DSA_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice || attr.device != dev) return DSA_ERR_INVALID_ARG;
+  }
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> g(g_static_mu);

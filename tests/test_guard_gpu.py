@@ -86,9 +86,13 @@ def decode_case(lens):
     return w, synth.decode_inputs(w, lengths=np.array(lens, dtype=np.int64))
 
 
-@pytest.mark.parametrize("want_indices", [True, False])
-def test_decode_writes_stay_inside_buffers(dsa, want_indices):
+@pytest.mark.parametrize("want_indices,zero_q", [(True, False), (False, False), (True, True)])
+def test_decode_writes_stay_inside_buffers(dsa, want_indices, zero_q):
+    # zero_q: every score +0, so sequences longer than 8192 rows take the
+    # select's many-candidate path (compaction in the workspace's key scratch)
     w, xd = decode_case([1, 2, 100, 2049, 9000, 70000])
+    if zero_q:
+        xd["q_idx"] = np.zeros_like(xd["q_idx"])
     t = {n: dev(xd[n]) for n in ("k_idx", "K", "V", "q_idx", "Q", "seq_start")}
     B, total, mx = xd["B"], int(xd["seq_start"][-1]), int(xd["lengths"].max())
     need = dsa.dsa_decode_workspace_size(B, total, w.d_idx, 0, w.H, w.D, w.top_k)
@@ -107,10 +111,13 @@ def test_decode_writes_stay_inside_buffers(dsa, want_indices):
     assert torch.equal(O.view(torch.int16), ref_o.view(torch.int16))
 
 
-def test_paged_decode_writes_stay_inside_buffers(dsa):
+@pytest.mark.parametrize("zero_q", [False, True])
+def test_paged_decode_writes_stay_inside_buffers(dsa, zero_q):
     w = synth.WORKLOADS["decode_64x128k"]
     lens = np.array([1, 2, 100, 2049, 9000, 70000], dtype=np.int64)
     xp = synth.paged_decode_inputs(w, lens, 16)
+    if zero_q:
+        xp["q_idx"] = np.zeros_like(xp["q_idx"])
     t = {n: dev(xp[n]) for n in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens",
                                  "q_idx", "Q")}
     B, mx = xp["B"], int(lens.max())

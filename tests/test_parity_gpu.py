@@ -3,8 +3,9 @@
 Bar: indices bit-exact (integer-valued indexer inputs make every score exact
 on both sides); attention outputs within max-abs 2e-2 of the oracle's FP64
 result rounded to BF16.  Small cases compare every row; the full-size
-workloads compare sampled rows (first rows, tile and capacity boundaries,
-the last rows, and a seeded random spread) and check properties of all rows.
+workloads compare every row at 32K and, at 64K and 128K, the first rows,
+tile and capacity boundaries, the last rows and 2048 seeded random rows, and
+check properties of all rows.
 """
 import numpy as np
 import pytest
@@ -259,7 +260,7 @@ def test_prefill_workload_4k_all_rows(dsa):
 
 # ------------------------------------------------------------------ prefill, full size
 
-def sampled_rows(L, k, n=48, seed=0):
+def sampled_rows(L, k, n=2048, seed=0):
     rng = np.random.default_rng(seed)
     fixed = [0, 1, 127, 128, k - 2, k - 1, k, k + 1, 2 * k, 4 * k, L // 2, L - 129, L - 128, L - 2, L - 1]
     rows = np.concatenate([np.array([r for r in fixed if 0 <= r < L]), rng.integers(0, L, n)])
@@ -292,13 +293,17 @@ def host_copy(x):
     return out
 
 
-@pytest.mark.parametrize("name", ["prefill_32k", "prefill_64k", "prefill_128k"])
-def test_prefill_full_workloads_sampled(dsa, name):
+@pytest.mark.parametrize("name,every_row", [("prefill_32k", True), ("prefill_64k", False),
+                                            ("prefill_128k", False)])
+def test_prefill_full_workloads(dsa, name, every_row):
+    """The full-size workloads: every row of the 32K one against the oracle;
+    at 64K and 128K the fixed boundary rows plus 2048 seeded random rows (the
+    oracle runs on every host thread), and properties of every row."""
     w = synth.WORKLOADS[name]
     x = host_copy(synth.prefill_inputs_torch(w, device="cuda"))
     idx, O, stats = run_prefill(dsa, x, w.top_k)
     check_index_properties(idx, w.top_k)
-    rows = sampled_rows(w.L, w.top_k)
+    rows = None if every_row else sampled_rows(w.L, w.top_k)
     compare(x, w.idx_dtype, w.top_k, idx, O, rows=rows)
     assert stats["fallback_rows"] < w.L // 100, stats
 
@@ -383,6 +388,66 @@ def test_decode_full_workload(dsa):
     assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
 
 
+def tie_queries(B, d, mode):
+    """Decode queries whose scores tie widely: "zero" makes every score +0;
+    "e0" puts a single 1 in dimension 0, so a score is relu(k_idx[s, 0] * scale)
+    and takes one of nine values (about len/9 keys share each)."""
+    q = np.zeros((B, d), dtype=np.int64)
+    if mode == "e0":
+        q[:, 0] = 1
+    return synth.fp8_bytes_of_ints(q)
+
+
+def boundary_bin_count(xd, top_k, scale):
+    """Keys at or above the bin of each sequence's m-th best score, binning by
+    the top bits of the FP32 score (bits 30..20), as the decode select does:
+    above 8192 the select takes its many-candidate path."""
+    out = []
+    ss = xd["seq_start"]
+    q = synth_fp8_values(xd["q_idx"])
+    for b in range(len(ss) - 1):
+        k = synth_fp8_values(xd["k_idx"][ss[b]:ss[b + 1]])
+        sc = np.maximum(np.float32(k @ q[b]) * np.float32(scale), np.float32(0)).astype(np.float32)
+        bins = sc.view(np.uint32) >> 20
+        m = min(top_k, sc.size)
+        kth = np.sort(bins)[::-1][m - 1]
+        out.append(int((bins >= kth).sum()))
+    return out
+
+
+def synth_fp8_values(a):
+    # the test inputs are exact small integers: decode E4M3 codes of -4..4
+    table = {int(c): v for v, c in zip(range(-4, 5), synth.fp8_bytes_of_ints(np.arange(-4, 5)))}
+    lut = np.zeros(256, dtype=np.float64)
+    for c, v in table.items():
+        lut[c] = v
+    return lut[np.asarray(a)]
+
+
+@pytest.mark.parametrize("mode,lens", [
+    ("zero", [1, 5000, 8193, 20000, 131072]),
+    ("e0", [9000, 30000, 100000, 131072]),
+])
+def test_decode_wide_ties_many_candidates(dsa, mode, lens):
+    """Scores that tie across the k-th place on long sequences: more than 8192
+    keys fall in the boundary bin, so the select compacts its candidates in
+    global scratch and selects there; ties must still go to the lower index."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array(lens, dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    xd["q_idx"] = tie_queries(len(lens), w.d_idx, mode)
+    scale = oracle.default_index_scale(w.d_idx)
+    assert max(boundary_bin_count(xd, w.top_k, scale)) > 8192
+    idx, O = run_decode(dsa, xd, w.top_k)
+    ri, ro = oracle.decode(xd, w.idx_dtype, w.top_k)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+    if mode == "zero":
+        for b, n in enumerate(lens):
+            m = min(int(n), w.top_k)
+            assert idx[b, :m].tolist() == list(range(m))
+
+
 # ------------------------------------------------------------------ paged decode
 
 def run_decode_paged(dsa, xp, top_k, max_len=None):
@@ -410,6 +475,24 @@ def test_decode_paged_matches_oracle(dsa, block_size, idx_dtype, d, D, top_k):
     idx, O = run_decode_paged(dsa, xp, top_k)
     assert dsa.dsa_sync_status() == 0
     ri, ro = oracle.decode_paged(xp, idx_dtype, top_k)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    got = O.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL
+
+
+@pytest.mark.parametrize("mode", ["zero", "e0"])
+def test_decode_paged_wide_ties_many_candidates(dsa, mode):
+    """The wide-tie decode of test_decode_wide_ties_many_candidates over a
+    block-paged cache (blocks of 64 rows in seeded order)."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([3000, 20000, 131072], dtype=np.int64)
+    xp = synth.paged_decode_inputs(w, lens, 64)
+    xp["q_idx"] = tie_queries(len(lens), w.d_idx, mode)
+    c = dict(xp["contiguous"], q_idx=xp["q_idx"])
+    assert max(boundary_bin_count(c, w.top_k, oracle.default_index_scale(w.d_idx))) > 8192
+    idx, O = run_decode_paged(dsa, xp, w.top_k)
+    assert dsa.dsa_sync_status() == 0
+    ri, ro = oracle.decode_paged(xp, w.idx_dtype, w.top_k)
     assert np.array_equal(idx.cpu().numpy(), ri)
     got = O.view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL

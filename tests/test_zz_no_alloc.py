@@ -48,11 +48,49 @@ def test_static_scratch_decode_matches_workspace_decode_twice(dsa):
         assert err <= ATOL, f"call {call}: max-abs {err}"
 
 
+def small_batch(B=64, H=16, D=128, d=128):
+    """Real device buffers for a batch of B one-row sequences (seq_start = 0..B)."""
+    return {
+        "k_idx": torch.zeros((B, d), dtype=torch.uint8, device="cuda"),
+        "K": torch.zeros((B, D), dtype=torch.bfloat16, device="cuda"),
+        "V": torch.zeros((B, D), dtype=torch.bfloat16, device="cuda"),
+        "seq_start": torch.arange(B + 1, dtype=torch.int64, device="cuda"),
+        "q_idx": torch.zeros((B, d), dtype=torch.uint8, device="cuda"),
+        "Q": torch.zeros((B, H, D), dtype=torch.bfloat16, device="cuda"),
+        "O": torch.zeros((B, H, D), dtype=torch.bfloat16, device="cuda"),
+    }
+
+
 def test_static_scratch_rejects_sizes_beyond_its_block(dsa):
     import ctypes
     lib = dsa.load()
-    P = ctypes.c_void_p
     too_many_rows = 1 << 22
-    st = lib.dsa_decode_static(P(16), P(16), P(16), P(16), 64, too_many_rows, 131072, 0, 128, 128,
-                               P(16), P(16), 16, 2048, float("nan"), float("nan"), P(16), None, None)
+    # the size bound alone: such a call needs more scratch than the block holds
+    assert dsa.dsa_decode_workspace_size(64, too_many_rows, 128, 0, 16, 128, 2048) > (18 << 20)
+    # Every pointer is a real device buffer of a small batch, so even a call
+    # that got past the host-side size check would meet the device-side check
+    # (seq_start[B] != total_rows) and read nothing out of bounds.
+    t = small_batch()
+    st = lib.dsa_decode_static(*(ctypes.c_void_p(t[n].data_ptr()) for n in ("k_idx", "K", "V", "seq_start")),
+                               64, too_many_rows, 131072, 0, 128, 128,
+                               ctypes.c_void_p(t["q_idx"].data_ptr()), ctypes.c_void_p(t["Q"].data_ptr()),
+                               16, 2048, float("nan"), float("nan"), ctypes.c_void_p(t["O"].data_ptr()),
+                               None, None)
     assert st == 3   # DSA_ERR_WORKSPACE: the built-in scratch is too small for these sizes
+    assert dsa.dsa_sync_status() == 0   # nothing was enqueued
+
+
+def test_static_scratch_rejects_output_off_the_current_device(dsa):
+    # The block is per device: an output in host memory is refused before any launch.
+    t = small_batch()
+    O_host = torch.zeros((64, 16, 128), dtype=torch.bfloat16).pin_memory()
+    import ctypes
+    lib = dsa.load()
+    st = lib.dsa_decode_static(*(ctypes.c_void_p(t[n].data_ptr()) for n in ("k_idx", "K", "V", "seq_start")),
+                               64, 64, 1, 0, 128, 128,
+                               ctypes.c_void_p(t["q_idx"].data_ptr()), ctypes.c_void_p(t["Q"].data_ptr()),
+                               16, 2048, float("nan"), float("nan"), ctypes.c_void_p(O_host.data_ptr()),
+                               None, None)
+    assert st == 1   # DSA_ERR_INVALID_ARG
+    assert dsa.dsa_sync_status() == 0
+    assert bool((O_host == 0).all())
