@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the 4K/32K/64K prefill sub-lines")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample time")
     ap.add_argument("--workload", default=PREFILL,
                     choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k", "prefill_32k_bf16"],
@@ -72,6 +73,62 @@ def peaks():
     except (OSError, ValueError, KeyError):
         pass
     return p
+
+
+def measured_peaks_in_run(dev) -> dict:
+    """Tensor peaks measured in this run (CUDA events, best of 10): FP8 E4M3 with
+    torch._scaled_mm and BF16 with torch.matmul, both 8192^3 (2 N^3 FLOP), as a
+    burst on an idle GPU.  The FP8 figure is the denominator for the FP8
+    indexer; MEASURED_PEAKS.json holds no FP8 number."""
+    import torch
+    n = 8192
+    out = {}
+    a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    ab = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    bb = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    for name, fn in (("fp8_tflops", lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one,
+                                                              out_dtype=torch.bfloat16)),
+                     ("bf16_tflops", lambda: torch.matmul(ab, bb))):
+        for _ in range(3):
+            fn()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        out[name] = 2.0 * n ** 3 / (best / 1000.0) / 1e12
+    del a, b, ab, bb
+    torch.cuda.empty_cache()
+    out["how"] = "torch._scaled_mm FP8 E4M3 and torch.matmul BF16, 8192^3, best of 10 (burst)"
+    return out
+
+
+def gather_ceiling(dsa, idx, K, V, gather_bytes, stream) -> dict:
+    """Rate of dsa_gather_probe over the prefill's own indices: the attention's
+    exact K/V row reads into shared memory and nothing else, best of a few
+    launch shapes (CTAs per SM x 16 KB stages) and three launches each."""
+    import torch
+    best, shape = float("inf"), None
+    sink = torch.zeros(1, dtype=torch.int64, device=idx.device)
+    for cps, st in ((2, 3), (2, 6), (3, 4), (4, 3)):
+        dsa.dsa_gather_probe(idx, K, V, cps, st, sink=sink, stream=stream)
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dsa.dsa_gather_probe(idx, K, V, cps, st, sink=sink, stream=stream)
+            e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            if ms < best:
+                best, shape = ms, f"{cps} CTAs/SM x {st} stages of 16 KB"
+    return {"gbs": gather_bytes / (best / 1000.0) / 1e9, "ms": best, "shape": shape,
+            "how": "dsa_gather_probe: the attention's K and V rows (this step's indices) copied into "
+                   "shared memory with 16-byte cp.async and nothing else; best launch shape"}
 
 
 def reduce_max(x: float, world: int, device) -> float:
@@ -191,6 +248,69 @@ def decode_work(w, lengths):
     }
 
 
+def line_config(w, world: int) -> dict:
+    return {"workload": workload_desc(w), "parallelism": f"{world} independent sequences (one per GPU)",
+            "l2": "inputs larger than L2 (~9 GB touched per step vs 126 MB L2)"}
+
+
+def workload_desc(w) -> str:
+    return (f"{w.name}: L={w.L} causal, q_idx/k_idx [L,{w.d_idx}] {w.idx_dtype} ints in [-4,4]"
+            f"{' with local boost' if w.local_boost else ''}, Q [L,{w.H},{w.D}], K/V [L,{w.D}] bf16 N(0,1), "
+            f"top_k={w.top_k}")
+
+
+def time_prefill_config(dsa, synth, name, steps, warmup, dev, stream, seed, fp8_peak, bf16_peak, max_over_ranks):
+    """One prefill workload timed on its own: whole-call time (CUDA events over `steps`
+    calls after `warmup`), per-stage times from a second pass, indexer TFLOP/s against the
+    peak of its input dtype."""
+    import torch
+    w = synth.WORKLOADS[name]
+    x = synth.prefill_inputs_torch(w, seed=seed, device=dev)
+    idt = dsa.IDX_BF16 if w.idx_dtype == "bf16" else dsa.IDX_FP8_E4M3
+    ws = torch.empty(dsa.dsa_prefill_workspace_size(w.L, w.d_idx, idt, w.H, w.D, w.top_k),
+                     dtype=torch.uint8, device=dev)
+    idx = torch.empty((w.L, w.top_k), dtype=torch.int32, device=dev)
+    O = torch.empty((w.L, w.H, w.D), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        dsa.dsa_prefill(x["q_idx"], x["k_idx"], x["Q"], x["K"], x["V"], w.top_k, indices=idx, O=O,
+                        workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if dsa.dsa_sync_status(stream) != 0:
+        raise RuntimeError(f"device-side error in {name}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    dsa.dsa_stage_timing(True)
+    for _ in range(steps):
+        step()
+    torch.cuda.synchronize()
+    dsa.dsa_stage_timing(False)
+    st = {k_: v[0] / steps for k_, v in dsa.dsa_stage_times().items() if v[1] > 0}
+    work = prefill_work(w)
+    idx_ms = st.get("indexer_filter", float("nan"))
+    tflops = work["indexer_flops"] / (idx_ms / 1000.0) / 1e12
+    peak = fp8_peak if w.idx_dtype == "fp8" else bf16_peak
+    out = {"workload": workload_desc(w), "ms_per_step": ms, "queries_per_s": w.L / (ms / 1000.0),
+           "stage_ms": st,
+           "indexer": {"tflops": tflops, "dtype": w.idx_dtype, "peak": peak, "frac": tflops / peak,
+                       "frac_fp8_peak": tflops / fp8_peak, "flops_per_launch": work["indexer_flops"],
+                       "peak_source": "FP8 measured in this run" if w.idx_dtype == "fp8"
+                       else "BF16 burst, MEASURED_PEAKS.json"},
+           "attention_gather_gbs": work["gather_bytes"] / (st.get("attention", float("nan")) / 1000.0) / 1e9,
+           "select_stats": dsa.dsa_last_stats(ws, stream)}
+    del x, ws, idx, O
+    torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------------------- CPU oracle leg
 
 def cpu_oracle_sample(w, host, target_s, seed=0):
@@ -198,18 +318,27 @@ def cpu_oracle_sample(w, host, target_s, seed=0):
     until one run takes at least half of target_s; returns (queries/s, rows,
     seconds, threads) of that last run."""
     import oracle
-    threads = oracle.max_threads()
+    threads = host_threads()
     rng = np.random.default_rng(seed)
     n = max(4, 2 * threads)
     for _ in range(5):
         rows = np.sort(rng.choice(w.L, size=min(n, w.L), replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
+        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows, nthreads=threads)
         dt = time.perf_counter() - t0
         if dt >= 0.5 * target_s or len(rows) == w.L:
             break
         n = int(min(w.L, len(rows) * 0.9 * target_s / max(dt, 1e-3)))
     return len(rows) / dt, len(rows), dt, threads
+
+
+def host_threads() -> int:
+    """Host cores this process may run on (torchrun's OMP_NUM_THREADS=1 does not apply
+    to the oracle, which is given this count explicitly)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def host_copy(x):
@@ -232,21 +361,22 @@ def run_reference(args):
     if rank != 0:
         return
     w = synth.WORKLOADS[PREFILL]
+    world_n = max(1, args.gpus)
     host = synth.prefill_inputs(w)
     per_step = max(2.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
     # size one step's sample from a calibration run (untimed)
     import oracle
-    threads = oracle.max_threads()
+    threads = host_threads()
     probe = np.linspace(0, w.L - 1, max(4, threads), dtype=np.int64)
     t0 = time.perf_counter()
-    oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=probe)
+    oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=probe, nthreads=threads)
     n = int(max(len(probe), len(probe) * per_step / max(time.perf_counter() - t0, 1e-3)))
     rng = np.random.default_rng(1)
     times = []
     for step in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(w.L, size=n, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows)
+        oracle.prefill_rows(host, w.idx_dtype, w.top_k, rows=rows, nthreads=threads)
         if step >= args.warmup:
             times.append(time.perf_counter() - t0)
     total = sum(times)
@@ -256,9 +386,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{PREFILL}: L=131072 causal, q_idx/k_idx [L,160] bf16 ints in [-4,4], "
-                               f"Q [L,16,128], K/V [L,128] bf16 N(0,1), top_k=2048",
-                   "sample_rows_per_step": n},
+        "config": line_config(w, world_n),
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads, "kind": "oracle",
                          "sample": f"{n} random query rows of {PREFILL} per step (full work of each row)"},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -268,8 +396,28 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU leg
 
+def spawn_ranks(args) -> None:
+    """`--gpus N` outside torchrun: start N ranks on this node (one process per GPU,
+    rendezvous on 127.0.0.1) and exit with their status.  Under torchrun the
+    world size must equal N."""
+    if "WORLD_SIZE" in os.environ:
+        if int(os.environ["WORLD_SIZE"]) != args.gpus:
+            raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={os.environ['WORLD_SIZE']}")
+        return
+    if args.gpus <= 1:
+        return
+    import socket
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    raise SystemExit(subprocess.call(cmd))
+
+
 def main():
     args = parse()
+    spawn_ranks(args)
     rank, world, local = rank_info()
     if args.impl == "reference":
         run_reference(args)
@@ -296,6 +444,7 @@ def main():
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, world, dev)
 
+    run_peaks = measured_peaks_in_run(dev)
     w = synth.WORKLOADS[args.workload]
     seed = synth.SEED + rank              # every rank runs its own sequence
     x = synth.prefill_inputs_torch(w, seed=seed, device=dev)
@@ -352,13 +501,34 @@ def main():
     gather_gbs = work["gather_bytes"] / (att_ms / 1000.0) / 1e9
     dominant = max(("indexer_filter", "attention", "select", "indexer_sample", "threshold"),
                    key=lambda s: st_ms.get(s, 0.0))
-    # A contraction takes the peak of its own dtype: BF16 measured; FP8 = 2 x BF16 measured
-    # (the nominal dense FP8:BF16 ratio).  Sustained figures: the kernels run inside a long step.
-    idx_peak = pk["bf16_tflops_sustained"] * (2.0 if w.idx_dtype == "fp8" else 1.0)
-    fp8_peak = 2.0 * pk["bf16_tflops_sustained"]
+    # Peaks: HBM and BF16 from MEASURED_PEAKS.json (measured on this machine), FP8 measured in
+    # this run.  The stage kernels are timed one launch at a time inside a ~20 ms step, so the
+    # burst figures apply.
+    fp8_peak = run_peaks["fp8_tflops"]
+    bf16_peak = pk["bf16_tflops"]
+    idx_peak = fp8_peak if w.idx_dtype == "fp8" else bf16_peak
     indexer = {"tflops": indexer_tflops, "dtype": w.idx_dtype, "peak_own_dtype": idx_peak,
                "frac_own_dtype": indexer_tflops / idx_peak, "frac_fp8_peak": indexer_tflops / fp8_peak,
-               "flops_per_launch": work["indexer_flops"], "ms": idx_ms}
+               "flops_per_launch": work["indexer_flops"], "ms": idx_ms,
+               "peaks": f"own dtype: {'FP8 measured in this run' if w.idx_dtype == 'fp8' else 'BF16 burst, MEASURED_PEAKS.json'}; "
+                        f"FP8: measured in this run ({fp8_peak:.0f} TFLOP/s)"}
+    ceiling = gather_ceiling(dsa, idx, K, V, work["gather_bytes"], stream)
+    att_kernel = "attn_tc_kernel" if w.D == 128 else "attn_kernel"
+    att_src = "attention_tc.cu" if w.D == 128 else "attention.cu"
+    traffic = profiled_traffic(att_kernel, w.name, "sparse_attention_10_b200/csrc/" + att_src)
+    att_s = att_ms / 1000.0
+    att_gbs = work["gather_bytes"] / att_s / 1e9
+    attention = {
+        "kernel": att_kernel, "ms": att_ms,
+        "gather": {"achieved": att_gbs, "peak": ceiling["gbs"], "unit": "GB/s", "frac": att_gbs / ceiling["gbs"],
+                   "bytes_per_launch": work["gather_bytes"], "peak_source": ceiling["how"],
+                   "peak_shape": ceiling["shape"]},
+        "hbm": {"achieved": (traffic / att_s / 1e9) if traffic else None, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": (traffic / att_s / 1e9 / pk["hbm_gbs"]) if traffic else None,
+                "note": "DRAM bytes of one launch (ncu, profile summary) over this run's launch time"},
+        "tensor": {"achieved": work["attn_flops"] / att_s / 1e12, "peak": bf16_peak, "unit": "TFLOP/s",
+                   "frac": work["attn_flops"] / att_s / 1e12 / bf16_peak},
+    }
     if dominant.startswith("indexer"):
         flops = work["indexer_flops"] if dominant == "indexer_filter" else float("nan")
         ach = flops / (st_ms[dominant] / 1000.0) / 1e12
@@ -366,20 +536,24 @@ def main():
                 "unit": "TFLOP/s", "frac": ach / idx_peak,
                 "traffic": profiled_traffic("indexer_kernel", w.name, "sparse_attention_10_b200/csrc/indexer.cu")}
     elif dominant == "attention":
-        ach = work["attn_bytes"] / (st_ms["attention"] / 1000.0) / 1e9
-        att_kernel = "attn_tc_kernel" if w.D == 128 else "attn_kernel"
-        att_src = "attention_tc.cu" if w.D == 128 else "attention.cu"
-        roof = {"kernel": att_kernel, "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / pk["hbm_gbs"], "bytes_per_launch": work["attn_bytes"],
-                "note": "effective rate: the gathered K/V rows (algorithmic bytes) are mostly L2 hits, "
-                        "so it can exceed the HBM copy peak; DRAM traffic per launch is 'traffic'",
-                "traffic": profiled_traffic(att_kernel, w.name, "sparse_attention_10_b200/csrc/" + att_src)}
+        # The gathered K/V rows are random 256-byte rows of tensors that fit in L2: the kernel is
+        # bound by the rate the SMs can gather them, measured above by the probe on the same rows.
+        roof = {"kernel": att_kernel, "bound": "l2_gather", "achieved": att_gbs, "peak": ceiling["gbs"],
+                "unit": "GB/s", "frac": att_gbs / ceiling["gbs"], "bytes_per_launch": work["gather_bytes"],
+                "traffic": traffic,
+                "peak_source": "measured in this run: " + ceiling["how"],
+                "vs_hbm_copy_peak": {"peak": pk["hbm_gbs"], "frac": att_gbs / pk["hbm_gbs"],
+                                     "note": "algorithmic gather bytes over the HBM copy peak: above 1 "
+                                             "because K and V (67 MB) stay in L2"}}
     else:
         ach = (work["cand_bytes"] + 4.0 * w.L * w.top_k) / (st_ms[dominant] / 1000.0) / 1e9
         roof = {"kernel": "select_kernel", "bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": ach / pk["hbm_gbs"],
                 "traffic": profiled_traffic("select_kernel", w.name, "sparse_attention_10_b200/csrc/select.cu")}
-    roof["peak_source"] = pk["source"]
+    roof.setdefault("peak_source", pk["source"])
+    roof["traffic_source"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the profile "
+                              "summary in profiles/ whose recorded source hash matches this kernel's source "
+                              "(null when it does not)")
 
     # --- end to end through the public API with host buffers.  A serving loop
     # pipelines the transfers: while step i computes, step i+1's inputs go up
@@ -531,6 +705,18 @@ def main():
             "matches_contiguous": bool(torch.equal(idp, idd) and torch.equal(Op, Od))}
         del xp, wsp
 
+    # --- the other prefill workloads (4K, 32K and 64K), each timed on its own
+    configs = None
+    if not args.no_configs:
+        del idx, O
+        torch.cuda.empty_cache()
+        configs = {}
+        for name in ("prefill_4k", "prefill_32k", "prefill_64k"):
+            if name != w.name:
+                configs[name] = time_prefill_config(dsa, synth, name, max(5, args.steps // 2), args.warmup,
+                                                    dev, stream, seed, run_peaks["fp8_tflops"], pk["bf16_tflops"],
+                                                    max_over_ranks)
+
     # --- CPU oracle baseline (rank 0, one GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -546,13 +732,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if w.idx_dtype == "bf16" else "fp8 indexer / bf16 attention", "data": "synthetic",
-            "config": {"workload": f"{w.name}: L={w.L} causal, q_idx/k_idx [L,{w.d_idx}] {w.idx_dtype} ints "
-                                   f"in [-4,4]{' with local boost' if w.local_boost else ''}, "
-                                   f"Q [L,{w.H},{w.D}], K/V [L,{w.D}] bf16 N(0,1), top_k={w.top_k}",
-                       "parallelism": f"{world} independent sequences (one per GPU)",
-                       "l2": "inputs larger than L2 (~9 GB touched per step vs 126 MB L2)"},
+            "config": line_config(w, world),
             "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs, "indexer": indexer,
-            "stage_ms": st_ms, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "attention": attention, "stage_ms": st_ms, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "peaks_in_run": run_peaks, "configs": configs,
             "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clocks.summary(),
             "decode": decode, "select_stats": stats,
         }

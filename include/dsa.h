@@ -234,6 +234,26 @@ dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
 dsa_status dsa_debug_force_fallback(int period);
 
 /*
+ * dsa_gather_probe — diagnostic: the memory ceiling of the attention's
+ * gather.  The attention of section 3.3 reads, for each query, the K and V
+ * rows of its kept keys (section 4.2: one K/V shared by every head), random
+ * rows that mostly hit in L2.  This call copies, for every query row t < L,
+ * the rows indices[t, 0 : min(t + 1, top_k)] of K and then of V into a
+ * shared-memory ring (16-byte asynchronous copies, stages of 16 KB) and does
+ * nothing else with them, on num_SMs * ctas_per_sm CTAs of 128 threads with
+ * `stages` stages each.  Timing it gives the rate at which this device
+ * gathers exactly the attention's rows.
+ *   indices  device [L, top_k] int32 (a dsa_prefill output); ids outside
+ *            [0, L) read row 0
+ *   K, V     device [L, D] BF16, D in {64, 128}, 16-byte aligned
+ *   sink     device, 8 bytes, may be written (keeps the loads live)
+ * ctas_per_sm in [1, 8]; stages in {2, 3, 4, 6}.
+ */
+dsa_status dsa_gather_probe(const int32_t* indices, int64_t L, int top_k, const void* K,
+                            const void* V, int D, int ctas_per_sm, int stages, uint64_t* sink,
+                            void* stream);
+
+/*
  * dsa_decode_static — dsa_decode for callers that cannot allocate device
  * memory: a plugin whose host application owns every device allocation, or
  * a serving loop that must not call cudaMalloc (it can synchronise the device

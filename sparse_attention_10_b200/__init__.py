@@ -19,7 +19,7 @@ __all__ = [
     "dsa_prefill_workspace_size", "dsa_prefill", "dsa_decode_workspace_size", "dsa_decode",
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "dsa_debug_force_fallback", "IDX_FP8_E4M3", "IDX_BF16",
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
-    "dsa_decode_paged_workspace_size", "dsa_decode_paged",
+    "dsa_decode_paged_workspace_size", "dsa_decode_paged", "dsa_gather_probe",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -62,6 +62,7 @@ def load() -> ctypes.CDLL:
         "dsa_decode_paged_workspace_size": ([I, I64, I, I, I, I, I], SZ),
         "dsa_decode_paged": ([P, P, P, I64, I, P, I, P, I, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ,
                               P], I),
+        "dsa_gather_probe": ([P, I64, I, P, P, I, I, I, P, P], I),
         "dsa_stage_timing": ([I], I),
         "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
     }
@@ -255,6 +256,19 @@ def dsa_decode_static(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq
                                _dev(indices, "indices") if indices is not None else None, _stream(stream))
     _check(st, "dsa_decode_static")
     return O, indices
+
+
+def dsa_gather_probe(indices: torch.Tensor, K: torch.Tensor, V: torch.Tensor, ctas_per_sm: int, stages: int,
+                     sink: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Diagnostic: gather the K and V rows listed in indices into shared memory
+    and nothing else (the memory ceiling of the attention's gather)."""
+    L, top_k = indices.shape
+    D = K.shape[1]
+    if sink is None:
+        sink = torch.zeros(1, dtype=torch.int64, device=indices.device)
+    _check(load().dsa_gather_probe(_dev(indices, "indices"), L, top_k, _dev(K, "K"), _dev(V, "V"), D,
+                                   int(ctas_per_sm), int(stages), _dev(sink, "sink"), _stream(stream)),
+           "dsa_gather_probe")
 
 
 def dsa_sync_status(stream=None) -> int:

@@ -88,4 +88,28 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_reference_arm_other_ranks_do_no_work():
-    assert _bench(["--impl", "reference", "--steps", "1", "--warmup", "0"], {"RANK": "1", "WORLD_SIZE": "2"}) == []
+    assert _bench(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"],
+                  {"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_bench_starts_its_own_ranks():
+    """`--gpus 2` outside torchrun starts two ranks itself (the reference arm needs no
+    GPU); exactly one line comes back, from rank 0, and it reports both ranks."""
+    clean = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK",
+                                                               "MASTER_ADDR", "MASTER_PORT")}
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], cwd=ROOT, env=clean, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2
+
+
+def test_bench_rejects_world_size_other_than_gpus():
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "4",
+                        "--steps", "1", "--warmup", "0"], cwd=ROOT, env=dict(os.environ, RANK="0", WORLD_SIZE="2"),
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
