@@ -115,7 +115,7 @@ def gather_ceiling(dsa, idx, K, V, gather_bytes, stream) -> dict:
     import torch
     best, shape = float("inf"), None
     sink = torch.zeros(1, dtype=torch.int64, device=idx.device)
-    for cps, st in ((2, 3), (2, 6), (3, 4), (4, 3)):
+    for cps, st in ((2, 3), (4, 3), (5, 2), (6, 2), (7, 2)):
         dsa.dsa_gather_probe(idx, K, V, cps, st, sink=sink, stream=stream)
         for _ in range(3):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

@@ -52,7 +52,7 @@ float default_scale(float s, int dim) {
 // ---- prefill workspace ----------------------------------------------------------
 
 struct PrefillPlan {
-  int cap_half;     // candidates kept per (row, column half)
+  int cap_part;     // candidates kept per (row, column part of the indexer tile)
   int cap_all;      // rows with t + 1 <= cap_all keep every key
   int target;       // candidates aimed for per row by the threshold
   int samp_ld;
@@ -68,8 +68,11 @@ PrefillPlan plan_prefill(int64_t L, int top_k) {
   // row) is a > 4-sigma event; each extra 0.1 k costs filter stores and
   // select work in proportion.
   p.target = (top_k * 7 + 2) / 5;
-  p.cap_half = ((top_k * 5 / 4 + 128) + 15) / 16 * 16;    // per half: 1.25 k + 128
-  p.cap_all = p.cap_half;  // rows kept whole must fit one column half
+  // Per part about target / kCandParts candidates arrive; the capacity leaves twice that plus
+  // 128.  Rows with t + 1 <= cap_all (1.25 k + 128) keep every key: at most
+  // ceil(cap_all / 256) * 256 / kCandParts of them fall in one part, below cap_part.
+  p.cap_part = ((top_k * 14 / (5 * kCandParts) + 128) + 15) / 16 * 16;
+  p.cap_all = ((top_k * 5 / 4 + 128) + 15) / 16 * 16;
   p.samp_ld = kSampTilesMax * kBN;
   p.fb_ctas = std::max(1, num_sms());
   size_t o = 0;
@@ -78,9 +81,9 @@ PrefillPlan plan_prefill(int64_t L, int top_k) {
   p.off_tau = o;
   o = align_up(o + L * sizeof(float));
   p.off_cand_n = o;
-  o = align_up(o + 2 * L * sizeof(int));
+  o = align_up(o + kCandParts * L * sizeof(int));
   p.off_cand = o;
-  o = align_up(o + static_cast<size_t>(2 * L) * p.cap_half * sizeof(unsigned long long));
+  o = align_up(o + static_cast<size_t>(kCandParts * L) * p.cap_part * sizeof(unsigned long long));
   p.off_samp = o;
   o = align_up(o + static_cast<size_t>(L) * p.samp_ld * sizeof(uint16_t));
   p.off_fb_rows = o;
@@ -422,7 +425,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   a.tau = tau;
   a.cand = cand;
   a.cand_n = cand_n;
-  a.cap = plan.cap_half;
+  a.cap = plan.cap_part;
   {
     StageScope scope(2, 1, s);
     if ((st = launch_indexer(a, s)) != DSA_OK) return st;
@@ -431,7 +434,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   SelectLaunch sl{};
   sl.L = L;
   sl.top_k = top_k;
-  sl.cap = plan.cap_half;
+  sl.cap = plan.cap_part;
   sl.cand = cand;
   sl.cand_n = cand_n;
   sl.tau = tau;

@@ -6,7 +6,7 @@
 // accumulate in tensor memory.  One CTA per SM, persistent over 128-query
 // tiles; for each tile it streams 256-key tiles through a TMA -> shared memory
 // ring, issues tcgen05.mma into one of two TMEM accumulators (128 lanes x 256
-// columns each) and lets eight epilogue warps read the other one.
+// columns each) and lets the epilogue warps read the other one.
 //
 // The epilogue never writes the L x L matrix (section 3.3 / 4.3: the
 // selection consumes scores where they are produced).  Three modes:
@@ -18,10 +18,14 @@
 // Causal: key tiles entirely above the diagonal are never issued; the
 // diagonal tile is masked per key in the epilogue.
 //
-// Warp roles (320 threads): warp 0 issues TMA, warp 1 owns TMEM and issues
-// MMAs (one lane), warps 2..9 are the epilogue.  Warp w reads TMEM lanes
-// 32*(w%4)..+31; warps 2..5 take columns 0..127 of a tile, 6..9 columns
-// 128..255.  Every wait is bounded; on timeout the CTA drains its own copies
+// Warp roles (64 + 128 * kCandParts threads): warp 0 issues TMA, warp 1 owns
+// TMEM and issues MMAs (one lane), the rest are the epilogue.  Warp w reads
+// TMEM lanes 32*(w%4)..+31 (the rule for tcgen05.ld) and columns part p =
+// (w-2)/4 of a tile (256 / kCandParts columns), so each query row has one
+// candidate list per column part, each in ascending key order.  Two parts
+// (eight epilogue warps) measured best over the whole step: four parts cut
+// the 128K filter from 5.85 to 5.14 ms but the select's four-way merge cost
+// 1.2 ms more.  Every wait is bounded; on timeout the CTA drains its own copies
 // and MMAs, frees TMEM and exits with DSA_ERR_TIMEOUT recorded.
 #include <cudaTypedefs.h>
 
@@ -34,8 +38,9 @@ namespace dsa {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 4 * kCandParts;   // four TMEM lane quarters x column parts
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kPartCols = kBN / kCandParts;  // columns of a tile one epilogue warp reads
 constexpr int kChunk = 16;        // columns per TMEM load in the epilogue
 constexpr int kMiscBytes = 1024;  // barriers, TMEM slot, abort flag
 constexpr int kSmemLimit = 227 * 1024;
@@ -74,7 +79,7 @@ struct Params {
   const float* tau;
   unsigned long long* cand;
   int* cand_n;
-  int cap;        // filter: per-half capacity; sample: full capacity (rows below are kept whole)
+  int cap;        // filter: per-part capacity; sample: full capacity (rows below are kept whole)
   uint16_t* samp;
   int samp_ld;
   float* scores;
@@ -326,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int half = ew >> 2;
+    const int part = ew >> 2;
     const int row_local = quarter * 32 + lane;
     uint32_t acc_it = 0;
     bool ok = true;
@@ -342,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.mode == kModeFilter && row_ok) tau = p.tau[t];
       int count = 0;
       unsigned long long* my_cand =
-          p.mode == kModeFilter && row_ok ? p.cand + (2 * t + half) * static_cast<int64_t>(p.cap)
+          p.mode == kModeFilter && row_ok ? p.cand + (kCandParts * t + part) * static_cast<int64_t>(p.cap)
                                           : nullptr;
       for (int j = 0; j < nt; ++j) {
         const uint32_t buf = acc_it & 1;
@@ -353,10 +358,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int kt = item_ktile(p, qt, j, nt);
         const uint32_t tbase =
-            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kBN + half * 128;
+            tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + buf * kBN + part * kPartCols;
         // Chunk c+1's TMEM load is in flight while chunk c is processed.
         auto process = [&](int c, uint32_t (&v)[kChunk]) {
-            const int64_t s0 = static_cast<int64_t>(kt) * kBN + half * 128 + c * kChunk;
+            const int64_t s0 = static_cast<int64_t>(kt) * kBN + part * kPartCols + c * kChunk;
             if (p.mode == kModeFilter) {
               uint32_t pass = 0;
 #pragma unroll
@@ -393,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int q = 0; q < kChunk / 2; ++q)
                   w[q] = sample_key16(v[2 * q]) | (sample_key16(v[2 * q + 1]) << 16);
-                uint4* dst = reinterpret_cast<uint4*>(p.samp + t * p.samp_ld + j * kBN + half * 128 +
+                uint4* dst = reinterpret_cast<uint4*>(p.samp + t * p.samp_ld + j * kBN + part * kPartCols +
                                                       c * kChunk);
                 dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
                 dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -416,15 +421,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld16(tbase, va);
         tmem_ld_wait_regs(va);
 #pragma unroll
-        for (int c = 0; c < 128 / kChunk; c += 2) {
+        for (int c = 0; c < kPartCols / kChunk; c += 2) {
           tmem_ld16(tbase + (c + 1) * kChunk, vb);
           process(c, va);
           __syncwarp();
           tmem_ld_wait_regs(vb);
-          if (c + 2 < 128 / kChunk) tmem_ld16(tbase + (c + 2) * kChunk, va);
+          if (c + 2 < kPartCols / kChunk) tmem_ld16(tbase + (c + 2) * kChunk, va);
           process(c + 1, vb);
           __syncwarp();
-          if (c + 2 < 128 / kChunk) tmem_ld_wait_regs(va);
+          if (c + 2 < kPartCols / kChunk) tmem_ld_wait_regs(va);
         }
         tc_fence_before();
         __syncwarp();
@@ -432,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++acc_it;
       }
       if (!ok) break;
-      if (p.mode == kModeFilter && row_ok) p.cand_n[2 * t + half] = count;
+      if (p.mode == kModeFilter && row_ok) p.cand_n[kCandParts * t + part] = count;
     }
   }
 

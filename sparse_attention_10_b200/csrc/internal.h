@@ -17,6 +17,7 @@ enum IndexerMode { kModeDense = 0, kModeSample = 1, kModeFilter = 2 };
 constexpr int kBM = 128;          // query rows per tile = TMEM lanes
 constexpr int kBN = 256;          // keys per tile = TMEM columns per accumulator
 constexpr int kSampTilesMax = 16; // key tiles sampled per query tile for the threshold
+constexpr int kCandParts = 2;     // candidate lists per query row: one per column part of a tile
 
 struct IndexerLaunch {
   const void* q_idx;

@@ -37,10 +37,11 @@ __global__ void __launch_bounds__(kProbeThreads) gather_probe_kernel(const int32
                                                                       const uint8_t* __restrict__ V,
                                                                       int row_bytes,
                                                                       unsigned long long* sink) {
+  constexpr int kPasses = 8;   // rows of a stage per thread: 64 rows of 256 B or 128 of 128 B
   extern __shared__ __align__(128) uint8_t ring[];
   const int lanes_per_row = row_bytes / 16;                     // 16 (D = 128) or 8 (D = 64)
-  const int rows_per_pass = kProbeThreads / lanes_per_row;
-  const int tile_rows = kProbeStage / row_bytes;                // 64 or 128
+  const int rows_per_pass = kProbeThreads / lanes_per_row;      // 8 or 16
+  const int tile_rows = rows_per_pass * kPasses;                // 64 or 128: one 16 KB stage
   const int sub = threadIdx.x % lanes_per_row, r0 = threadIdx.x / lanes_per_row;
   uint32_t acc = 0;
   uint32_t issued = 0;
@@ -48,27 +49,31 @@ __global__ void __launch_bounds__(kProbeThreads) gather_probe_kernel(const int32
     const int m = static_cast<int>(min64(t + 1, top_k));
     const int32_t* ids = idx + t * top_k;
     for (int j0 = 0; j0 < m; j0 += tile_rows) {
+      // the tile's row ids first (independent loads), then the copies
+      int64_t rows[kPasses];
+#pragma unroll
+      for (int u = 0; u < kPasses; ++u) {
+        const int j = j0 + r0 + u * rows_per_pass;
+        int64_t s = j < m ? __ldg(ids + j) : -1;
+        rows[u] = (s < 0 || s >= L) ? (j < m ? 0 : -1) : s;
+      }
+#pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint8_t* src = which ? V : K;
-        const uint32_t slot = issued % NST;
-        const uint32_t stage = smem_u32(ring + slot * kProbeStage);
-        for (int r = r0; r < tile_rows; r += rows_per_pass) {
-          const int j = j0 + r;
-          if (j < m) {
-            int64_t s = __ldg(ids + j);
-            s = (s < 0 || s >= L) ? 0 : s;
-            probe_cp16(stage + r * row_bytes + sub * 16, src + s * row_bytes + sub * 16);
-          }
-        }
+        const uint32_t stage = smem_u32(ring + (issued % NST) * kProbeStage);
+#pragma unroll
+        for (int u = 0; u < kPasses; ++u)
+          if (rows[u] >= 0)
+            probe_cp16(stage + (r0 + u * rows_per_pass) * row_bytes + sub * 16,
+                       src + rows[u] * row_bytes + sub * 16);
         asm volatile("cp.async.commit_group;" ::: "memory");
         ++issued;
         // The ring holds NST tiles.  With at most NST - 1 groups pending, the
         // tile in the slot the next copy reuses has landed: read one word of
         // this thread's own copies there before the slot is overwritten.
         probe_wait<NST - 1>();
-        const uint32_t next = issued % NST;
-        acc ^= *reinterpret_cast<const volatile uint32_t*>(ring + next * kProbeStage + r0 * row_bytes +
-                                                           sub * 16);
+        acc ^= *reinterpret_cast<const volatile uint32_t*>(ring + (issued % NST) * kProbeStage +
+                                                           r0 * row_bytes + sub * 16);
       }
     }
   }

@@ -3,10 +3,10 @@
 // Token selection of the DeepSeek Sparse Attention page (kwkr.cn/news/60693,
 // section 3.3): query t keeps min(top_k, t+1) keys ranked by (score desc,
 // key index asc).  The indexer stores each candidate as the 64-bit word
-// (raw accumulator bits << 32) | (0xFFFFFFFF - s), in two lists per row (one
-// per column half of its tile), each in ascending key order.
+// (raw accumulator bits << 32) | (0xFFFFFFFF - s), in kCandParts lists per
+// row (one per column part of its tile), each in ascending key order.
 //
-// select_kernel: one CTA per row.  The two lists are merged into one
+// select_kernel: one CTA per row.  The lists are merged into one
 // ascending-key run of sort keys: relu(acc) when that orders exactly like
 // the score relu(fp32(acc) * scale) (checked per row), else the score word
 // (non-negative, so its bits order like the value).  Stable LSD radix passes
@@ -143,9 +143,11 @@ __device__ void finish_row(KeyPtr keys, int n, int m, int top_k, int32_t* out,
 
 // ---- sort-based select of one row ----------------------------------------------------
 //
-// The filter writes each row's candidates as two lists (one per column half
-// of the indexer tile), each already in ascending key order.  The select
-// merges them into one ascending-index run, then sorts it by key with
+// The filter writes each row's candidates as kCandParts lists (one per
+// column part of the indexer tile), each already in ascending key order.
+// The select merges them into one ascending-index run (pairwise merge
+// paths: lists 0+1 and 2+3 side by side, then the two results), then sorts
+// it by key with
 // stable LSD counting passes (descending digit), so equal keys keep
 // ascending index: the result is the (score desc, index asc) order, and the
 // first m entries are the answer.  Only the span of key bits that differ
@@ -204,6 +206,30 @@ __device__ __forceinline__ KeyStats stats_read(const uint32_t* misc) {
   return KeyStats{misc[0], misc[1], misc[2], static_cast<int>(misc[3])};
 }
 
+// Merge two ascending-index runs of 64-bit candidate keys a[0, na) and
+// b[0, nb) into out[0, na + nb), threads tid < nthr of the block taking equal
+// slices of the output (merge path: each finds its split by binary search).
+__device__ void merge_keys_by_index(const unsigned long long* a, int na, const unsigned long long* b,
+                                    int nb, unsigned long long* out, int tid, int nthr) {
+  const int n = na + nb;
+  const int per = (n + nthr - 1) / nthr;
+  const int p0 = min(n, tid * per), p1 = min(n, p0 + per);
+  if (p0 >= p1) return;
+  int lo = max(0, p0 - nb), hi = min(p0, na);
+  while (lo < hi) {  // smallest i such that a[i] does not precede b[p0 - i - 1]
+    const int i = (lo + hi) >> 1;
+    if (key_index(a[i]) < key_index(b[p0 - i - 1]))
+      lo = i + 1;
+    else
+      hi = i;
+  }
+  int i = lo, j = p0 - lo;
+  for (int p = p0; p < p1; ++p) {
+    const bool take_a = j >= nb || (i < na && key_index(a[i]) < key_index(b[j]));
+    out[p] = take_a ? a[i++] : b[j++];
+  }
+}
+
 // Merge two ascending-index runs a[0, na) and b[0, nb) (64-bit candidate
 // keys) into one ascending-index run, written as relu(accumulator) words `sc`
 // and key indices `ix` (merge path: each thread finds its split by binary
@@ -256,13 +282,18 @@ struct SelParams {
   int force_fb_period;
 };
 
+// Two regions of 8 * kSortCap bytes.  Region 1 first holds the candidate
+// lists as loaded (raw), then the merged score words sc0 and key indices ix;
+// region 2 holds the first-level merges (tmp), then the sort's scratch sc1,
+// ps0, ps1.  With two lists they are loaded into region 2 and merged once.
 struct SelSmem {
-  unsigned long long* raw;  // [kSortCap] candidate keys; after the merge the same bytes
-  uint32_t* sc1;            //   hold sc1 [kSortCap], ps0 [kSortCap], ps1 [kSortCap]
+  unsigned long long* raw;  // region 1: [kSortCap] candidate keys
+  unsigned long long* tmp;  // region 2: [kSortCap] keys of the first-level merges
+  uint32_t* sc1;            // region 2 after the merge: sc1 [kSortCap], ps0, ps1 [kSortCap]
   uint16_t* ps0;
   uint16_t* ps1;
-  uint32_t* sc0;            // [kSortCap] score words
-  uint32_t* ix;             // [kSortCap] key indices
+  uint32_t* sc0;            // region 1 after the merge: [kSortCap] score words
+  uint32_t* ix;             //   and [kSortCap] key indices
   uint32_t* cnt;            // [warps][256] words: 16-bit radix counters [warps][512] / bitmap
   uint32_t* base;           // [512 + warps]
   uint32_t* misc;           // [8]
@@ -273,12 +304,13 @@ constexpr size_t kSelSmemBytes =
 __device__ __forceinline__ SelSmem carve_sel_smem(unsigned long long* smem) {
   SelSmem sm;
   sm.raw = smem;
-  sm.sc1 = reinterpret_cast<uint32_t*>(smem);
+  sm.tmp = smem + kSortCap;
+  sm.sc0 = reinterpret_cast<uint32_t*>(sm.raw);
+  sm.ix = sm.sc0 + kSortCap;
+  sm.sc1 = reinterpret_cast<uint32_t*>(sm.tmp);
   sm.ps0 = reinterpret_cast<uint16_t*>(sm.sc1 + kSortCap);
   sm.ps1 = sm.ps0 + kSortCap;
-  sm.sc0 = reinterpret_cast<uint32_t*>(smem + kSortCap);
-  sm.ix = sm.sc0 + kSortCap;
-  sm.cnt = sm.ix + kSortCap;
+  sm.cnt = reinterpret_cast<uint32_t*>(smem + 2 * kSortCap);
   sm.base = sm.cnt + kSortWarps * 256;
   sm.misc = sm.base + 512 + kSortWarps;
   return sm;
@@ -369,14 +401,22 @@ __device__ void sort_emit(const SelSmem& sm, int n, int m, bool zero_mode, int64
 __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams p) {
   extern __shared__ unsigned long long sel_smem[];
   const SelSmem sm = carve_sel_smem(sel_smem);
-  unsigned long long* raw = sm.raw;
   const int lane = threadIdx.x & 31;
+  static_assert(kCandParts == 2 || kCandParts == 4, "two or four candidate lists per row");
+  unsigned long long* lists = kCandParts == 4 ? sm.raw : sm.tmp;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
     const int m = static_cast<int>(min64(p.top_k, t + 1));
-    const int n0 = p.cand_n[2 * t], n1 = p.cand_n[2 * t + 1];
-    const bool overflow = n0 > p.cap || n1 > p.cap || n0 + n1 > kSortCap;
+    int nl[kCandParts];
+    int n = 0;
+    bool overflow = false;
+#pragma unroll
+    for (int q = 0; q < kCandParts; ++q) {
+      nl[q] = p.cand_n[kCandParts * t + q];
+      overflow |= nl[q] > p.cap;
+      n += nl[q];
+    }
+    overflow |= n > kSortCap;
     const bool zero_mode = __float_as_uint(p.tau[t]) == kZeroModeTauBits;
-    const int n = n0 + n1;
     const bool forced = p.force_fb_period > 0 && t % p.force_fb_period == 0;
     if (overflow || forced || (!zero_mode && n < m)) {
       if (threadIdx.x == 0) {
@@ -387,16 +427,36 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
       continue;
     }
     if (threadIdx.x == 0) atomicAdd(&p.counters[2], n);
-    const unsigned long long* c0 = p.cand + 2 * t * static_cast<int64_t>(p.cap);
-    const unsigned long long* c1 = c0 + p.cap;
-    // Both lists in flight at once (8-byte asynchronous copies), one wait.
+    const unsigned long long* c0 = p.cand + kCandParts * t * static_cast<int64_t>(p.cap);
+    // Every list in flight at once (8-byte asynchronous copies), one wait.
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const unsigned long long* src = i < n0 ? c0 + i : c1 + (i - n0);
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(raw + i)), "l"(src)
+      int q = 0, off = i;
+#pragma unroll
+      for (int r = 0; r + 1 < kCandParts; ++r)
+        if (q == r && off >= nl[r]) {
+          off -= nl[r];
+          q = r + 1;
+        }
+      const unsigned long long* src = c0 + q * static_cast<int64_t>(p.cap) + off;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(lists + i)), "l"(src)
                    : "memory");
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
+    // First level (four lists): 0+1 and 2+3 into region 2, half the block each.
+    int na = nl[0], nb = n - nl[0];
+    if (kCandParts == 4) {
+      const int half = blockDim.x / 2;
+      na = nl[0] + nl[1];
+      nb = n - na;
+      if (threadIdx.x < half)
+        merge_keys_by_index(lists, nl[0], lists + nl[0], nl[1], sm.tmp, threadIdx.x, half);
+      else
+        merge_keys_by_index(lists + na, nl[2], lists + na + nl[2], nl[kCandParts - 1], sm.tmp + na,
+                            threadIdx.x - half, half);
+      __syncthreads();
+    }
+    const unsigned long long* runs = kCandParts == 4 ? sm.tmp : lists;
     if (threadIdx.x == 0) {
       stats_init(sm.misc);
       sm.misc[4] = 0u;           // largest exponent field of a positive accumulator
@@ -404,7 +464,7 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
     }
     __syncthreads();
     uint32_t lo = 0xFFFFFFFFu, hi = 0u, orr = 0u, pos = 0u, emax = 0u, pmin = 0xFFFFFFFFu;
-    merge_by_index(raw, n0, raw + n0, n1, sm.sc0, sm.ix, lo, hi, orr, pos, emax, pmin);
+    merge_by_index(runs, na, runs + na, nb, sm.sc0, sm.ix, lo, hi, orr, pos, emax, pmin);
     stats_reduce(lo, hi, orr, pos, sm.misc);
     emax = __reduce_max_sync(0xFFFFFFFFu, emax);
     pmin = __reduce_min_sync(0xFFFFFFFFu, pmin);
@@ -708,7 +768,6 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
 
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
-  if (2 * a.cap > kSortCap) return DSA_ERR_UNSUPPORTED;
   SelParams p{a.L,      a.top_k,   a.cap,     a.scale,    a.cand,
               a.cand_n, a.tau,     a.indices, a.fb_rows,  a.counters, a.force_fb_period};
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
