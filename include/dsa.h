@@ -116,6 +116,35 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
                        int H, int D, float attn_scale, int top_k, int32_t* indices, void* O,
                        void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace dsa_prefill_chunk needs for Lq queries against Lk keys. */
+size_t dsa_prefill_chunk_workspace_size(int64_t Lq, int64_t Lk, int d_idx, int idx_dtype, int H,
+                                        int D, int top_k);
+
+/*
+ * dsa_prefill_chunk — dsa_prefill for the last Lq positions of a causal
+ * sequence of Lk tokens: the same three stages (sections 3.2, 3.3, 4.1-4.2)
+ * for query rows that sit at key positions Lk - Lq .. Lk - 1.  Query row i
+ * (position p = Lk - Lq + i) sees keys 0 .. p, keeps min(top_k, p + 1) of
+ * them, and its indices are key positions.  With Lq = Lk this is
+ * dsa_prefill.  It serves chunked prefill (a long prompt in pieces, each
+ * chunk against every key before it), several new tokens of one sequence at
+ * once (speculative or multi-token decode over a contiguous cache), and a
+ * split of one sequence's query rows over GPUs (each GPU runs its chunks
+ * against the key prefix they need).
+ *   q_idx    device [Lq, d_idx]   index rows of the queries
+ *   k_idx    device [Lk, d_idx]   index rows of all keys 0 .. Lk - 1
+ *   Q        device [Lq, H, D] BF16;  K, V  device [Lk, D] BF16
+ *   indices  device [Lq, top_k] int32, written (-1 padded)
+ *   O        device [Lq, H, D] BF16, written
+ *   workspace >= dsa_prefill_chunk_workspace_size(Lq, Lk, ...) bytes
+ * Limits as dsa_prefill, and 1 <= Lq <= Lk.
+ */
+dsa_status dsa_prefill_chunk(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                             float idx_scale, const void* Q, const void* K, const void* V,
+                             int64_t Lq, int64_t Lk, int H, int D, float attn_scale, int top_k,
+                             int32_t* indices, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
 /* Bytes of device workspace dsa_decode needs.  total_rows = sum of lengths. */
 size_t dsa_decode_workspace_size(int B, int64_t total_rows, int d_idx, int idx_dtype, int H,
                                  int D, int top_k);

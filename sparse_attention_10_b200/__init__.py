@@ -20,6 +20,7 @@ __all__ = [
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "dsa_debug_force_fallback", "IDX_FP8_E4M3", "IDX_BF16",
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
     "dsa_decode_paged_workspace_size", "dsa_decode_paged", "dsa_gather_probe",
+    "dsa_prefill_chunk_workspace_size", "dsa_prefill_chunk",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -52,6 +53,8 @@ def load() -> ctypes.CDLL:
         "dsa_indexer_scores": ([P, P, I, I, F, I64, I64, P, P], I),
         "dsa_prefill_workspace_size": ([I64, I, I, I, I, I], SZ),
         "dsa_prefill": ([P, P, I, I, F, P, P, P, I64, I, I, F, I, P, P, P, SZ, P], I),
+        "dsa_prefill_chunk_workspace_size": ([I64, I64, I, I, I, I, I], SZ),
+        "dsa_prefill_chunk": ([P, P, I, I, F, P, P, P, I64, I64, I, I, F, I, P, P, P, SZ, P], I),
         "dsa_decode_workspace_size": ([I, I64, I, I, I, I, I], SZ),
         "dsa_decode": ([P, P, P, P, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ, P], I),
         "dsa_sync_status": ([P], I),
@@ -153,6 +156,39 @@ def dsa_prefill(q_idx: torch.Tensor, k_idx: torch.Tensor, Q: torch.Tensor, K: to
                          _dev(indices, "indices"), _dev(O, "O"), _dev(workspace, "workspace"),
                          workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "dsa_prefill")
+    return indices, O
+
+
+def dsa_prefill_chunk_workspace_size(Lq: int, Lk: int, d_idx: int, idx_dtype: int, H: int, D: int,
+                                     top_k: int) -> int:
+    return int(load().dsa_prefill_chunk_workspace_size(Lq, Lk, d_idx, idx_dtype, H, D, top_k))
+
+
+def dsa_prefill_chunk(q_idx: torch.Tensor, k_idx: torch.Tensor, Q: torch.Tensor, K: torch.Tensor,
+                      V: torch.Tensor, top_k: int, idx_scale: Optional[float] = None,
+                      attn_scale: Optional[float] = None, indices: Optional[torch.Tensor] = None,
+                      O: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """DSA for the last Lq positions of a causal sequence of Lk = k_idx.shape[0] tokens
+    (query row i at key position Lk - Lq + i) -> (indices [Lq, top_k], O [Lq, H, D])."""
+    lib = load()
+    Lq, d = q_idx.shape
+    Lk = k_idx.shape[0]
+    _, H, D = Q.shape
+    idt = _idx_dtype(q_idx)
+    dev = q_idx.device
+    if indices is None:
+        indices = torch.empty((Lq, top_k), dtype=torch.int32, device=dev)
+    if O is None:
+        O = torch.empty((Lq, H, D), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(dsa_prefill_chunk_workspace_size(Lq, Lk, d, idt, H, D, top_k),
+                                dtype=torch.uint8, device=dev)
+    st = lib.dsa_prefill_chunk(_dev(q_idx, "q_idx"), _dev(k_idx, "k_idx"), idt, d, _scale(idx_scale),
+                               _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), Lq, Lk, H, D, _scale(attn_scale),
+                               top_k, _dev(indices, "indices"), _dev(O, "O"), _dev(workspace, "workspace"),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "dsa_prefill_chunk")
     return indices, O
 
 

@@ -88,6 +88,7 @@ struct AttnParams {
   const int* invalid;
   const int32_t* block_table;   // paged decode cache, else null
   int bt_ld, bs_log2;
+  int64_t q0;                   // prefill: query q sits at key position q0 + q
 };
 
 template <int D>
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       row_base = p.seq_start[q];
       count = static_cast<int>(min64(p.top_k, p.seq_start[q + 1] - row_base));
     } else {
-      count = static_cast<int>(min64(p.top_k, q + 1));
+      count = static_cast<int>(min64(p.top_k, p.q0 + q + 1));
     }
     const int per = (count + p.nsplit - 1) / p.nsplit;
     const int begin = min(count, sp * per), end = min(count, begin + per);
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     const int32_t* ids = p.idx + q * p.ld_idx + begin;
     // rows a query may read: its causal prefix (prefill) or its sequence (decode)
     const int row_limit = p.seq_start ? static_cast<int>(p.seq_start[q + 1] - row_base)
-                                      : static_cast<int>(min64(q + 1, 0x7FFFFFFF));
+                                      : static_cast<int>(min64(p.q0 + q + 1, 0x7FFFFFFF));
     // a paged cache's key rows are absolute (translated below)
     const int64_t kv_base = p.block_table ? 0 : row_base;
     const __nv_bfloat16* Kb = p.K + kv_base * D;
@@ -392,7 +393,7 @@ template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p{a.Q,      a.K,    a.V,       a.idx,         a.ld_idx, a.nq,
                a.H,      a.scale_log2, a.top_k, a.seq_start, a.nsplit, a.O,
-               a.part,   a.invalid, a.block_table, a.bt_ld, a.bs_log2};
+               a.part,   a.invalid, a.block_table, a.bt_ld, a.bs_log2, a.q0};
   const size_t smem = AttnSmem<D>::kBytes;
   static_assert(AttnSmem<D>::kStages * 2 * AttnSmem<D>::kTile >=
                     (4 * 16 * 2 + 4 * 16 * AttnSmem<D>::kMergeRow) * 4,

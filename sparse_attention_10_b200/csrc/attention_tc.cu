@@ -86,6 +86,7 @@ struct TcParams {
   float* part;
   const int* invalid;
   uint64_t limit_ns;
+  int64_t q0;          // prefill: query q sits at key position q0 + q
 };
 
 struct Item {
@@ -109,8 +110,8 @@ __device__ __forceinline__ Item make_item(const TcParams& p, int64_t item) {
     it.row_limit = static_cast<int>(min64(len, 0x7FFFFFFF));
   } else {
     it.row_base = 0;
-    count = static_cast<int>(min64(p.top_k, it.q + 1));
-    it.row_limit = static_cast<int>(min64(it.q + 1, 0x7FFFFFFF));
+    count = static_cast<int>(min64(p.top_k, p.q0 + it.q + 1));
+    it.row_limit = static_cast<int>(min64(p.q0 + it.q + 1, 0x7FFFFFFF));
   }
   const int per = (count + p.nsplit - 1) / p.nsplit;
   const int begin = min(count, it.sp * per), end = min(count, begin + per);
@@ -600,7 +601,7 @@ bool attention_tc_supported(const AttnLaunch& a) { return a.D == kD && a.H >= 1 
 dsa_status launch_attention_tc(const AttnLaunch& a, cudaStream_t stream) {
   TcParams p{a.Q,         a.K,      a.V,       a.idx, a.ld_idx,  a.nq,     a.H,
              a.scale_log2, a.top_k, a.seq_start, a.nsplit, a.O, a.part, a.invalid,
-             wait_limit_ns()};
+             wait_limit_ns(), a.q0};
   static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);

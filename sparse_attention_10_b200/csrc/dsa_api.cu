@@ -61,7 +61,8 @@ struct PrefillPlan {
       off_fb_hist, off_fb_slow, total;
 };
 
-PrefillPlan plan_prefill(int64_t L, int top_k) {
+// L query rows against Lk key rows (Lk = L for a whole sequence).
+PrefillPlan plan_prefill(int64_t L, int top_k, int64_t Lk) {
   PrefillPlan p{};
   // 1.4 k: on the synthetic workloads the realized count has a spread of
   // about 0.1 k around the target, so fewer than k survivors (a fallback
@@ -89,7 +90,7 @@ PrefillPlan plan_prefill(int64_t L, int top_k) {
   p.off_fb_rows = o;
   o = align_up(o + L * sizeof(int));
   p.off_fb_scratch = o;
-  o = align_up(o + static_cast<size_t>(p.fb_ctas) * L * sizeof(unsigned long long));
+  o = align_up(o + static_cast<size_t>(p.fb_ctas) * Lk * sizeof(unsigned long long));
   p.off_fb_hist = o;
   o = align_up(o + static_cast<size_t>(p.fb_ctas) * 4096 * sizeof(unsigned int));
   p.off_fb_slow = o;
@@ -364,25 +365,43 @@ dsa_status dsa_indexer_scores(const void* q_idx, const void* k_idx, int idx_dtyp
 size_t dsa_prefill_workspace_size(int64_t L, int d_idx, int idx_dtype, int H, int D, int top_k) {
   (void)d_idx; (void)idx_dtype; (void)H; (void)D;
   if (L < 1 || top_k < 1) return 0;
-  return plan_prefill(L, top_k).total;
+  return plan_prefill(L, top_k, L).total;
+}
+
+size_t dsa_prefill_chunk_workspace_size(int64_t Lq, int64_t Lk, int d_idx, int idx_dtype, int H,
+                                        int D, int top_k) {
+  (void)d_idx; (void)idx_dtype; (void)H; (void)D;
+  if (Lq < 1 || Lk < Lq || top_k < 1) return 0;
+  return plan_prefill(Lq, top_k, Lk).total;
 }
 
 dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
                        float idx_scale, const void* Q, const void* K, const void* V, int64_t L,
                        int H, int D, float attn_scale, int top_k, int32_t* indices, void* O,
                        void* workspace, size_t workspace_bytes, void* stream) {
+  return dsa_prefill_chunk(q_idx, k_idx, idx_dtype, d_idx, idx_scale, Q, K, V, L, L, H, D,
+                           attn_scale, top_k, indices, O, workspace, workspace_bytes, stream);
+}
+
+dsa_status dsa_prefill_chunk(const void* q_idx, const void* k_idx, int idx_dtype, int d_idx,
+                             float idx_scale, const void* Q, const void* K, const void* V,
+                             int64_t Lq, int64_t Lk, int H, int D, float attn_scale, int top_k,
+                             int32_t* indices, void* O, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   if (!q_idx || !k_idx || !Q || !K || !V || !indices || !O || !workspace) return DSA_ERR_INVALID_ARG;
   for (const void* ptr : {q_idx, k_idx, Q, K, V, static_cast<const void*>(indices),
                           static_cast<const void*>(O)})
     if (!aligned16(ptr)) return DSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return DSA_ERR_INVALID_ARG;
-  if (L < 1 || L > (int64_t(1) << 31) - 1) return DSA_ERR_INVALID_ARG;
+  if (Lq < 1 || Lk < Lq || Lk > (int64_t(1) << 31) - 1) return DSA_ERR_INVALID_ARG;
   if (top_k < 1 || top_k > DSA_MAX_TOP_K) return DSA_ERR_INVALID_ARG;
   if (H < 1 || H > DSA_MAX_HEADS) return DSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return DSA_ERR_UNSUPPORTED;
   dsa_status st = check_index_dims(idx_dtype, d_idx);
   if (st != DSA_OK) return st;
-  const PrefillPlan plan = plan_prefill(L, top_k);
+  const int64_t L = Lq;
+  const int64_t q0 = Lk - Lq;   // query row t sits at key position q0 + t
+  const PrefillPlan plan = plan_prefill(L, top_k, Lk);
   if (workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -405,10 +424,11 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   a.esize = es;
   a.d = d_idx;
   a.Lq = L;
-  a.Lk = L;
+  a.Lk = Lk;
+  a.q0 = q0;
   a.scale = iscale;
   a.limit_ns = wait_limit_ns();
-  if (L > plan.cap_all) {
+  if (Lk > plan.cap_all) {   // some row (the last, at position Lk - 1) needs a threshold
     StageScope scope(0, 1, s);
     a.mode = kModeSample;
     a.samp = samp;
@@ -418,7 +438,7 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   }
   {
     StageScope scope(1, 1, s);
-    st = launch_tau_select(samp, plan.samp_ld, L, plan.cap_all, plan.target, iscale, tau, s);
+    st = launch_tau_select(samp, plan.samp_ld, L, q0, plan.cap_all, plan.target, iscale, tau, s);
     if (st != DSA_OK) return st;
   }
   a.mode = kModeFilter;
@@ -433,6 +453,8 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
 
   SelectLaunch sl{};
   sl.L = L;
+  sl.q0 = q0;
+  sl.Lk = Lk;
   sl.top_k = top_k;
   sl.cap = plan.cap_part;
   sl.cand = cand;
@@ -460,7 +482,8 @@ dsa_status dsa_prefill(const void* q_idx, const void* k_idx, int idx_dtype, int 
   at.Q = static_cast<const __nv_bfloat16*>(Q);
   at.K = static_cast<const __nv_bfloat16*>(K);
   at.V = static_cast<const __nv_bfloat16*>(V);
-  at.kv_rows = L;
+  at.kv_rows = Lk;
+  at.q0 = q0;
   at.idx = indices;
   at.ld_idx = top_k;
   at.nq = L;

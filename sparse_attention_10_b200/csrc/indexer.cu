@@ -70,6 +70,7 @@ struct Maps {                // tensor maps per swizzle kind
 struct Params {
   const void* k_idx;
   int64_t Lq, Lk;
+  int64_t q0;     // causal modes: query row i sits at key position q0 + i
   int nkb, stages;
   Slices sl;
   uint32_t off_b, off_bar;
@@ -96,9 +97,9 @@ __device__ __forceinline__ int64_t item_qtile(const Params& p, int item) {
   return p.mode == kModeDense ? item : nqt - 1 - item;
 }
 
-__device__ __forceinline__ int64_t sample_span(int64_t qt) {
-  // Key tiles entirely below the band of 128 positions before the query tile.
-  const int64_t r0 = qt * kBM;
+__device__ __forceinline__ int64_t sample_span(int64_t r0) {
+  // Key tiles entirely below the band of 128 positions before the query tile
+  // whose first row sits at key position r0.
   return r0 >= 128 ? (r0 - 128) / kBN : 0;
 }
 
@@ -106,16 +107,16 @@ __device__ __forceinline__ int item_ntiles(const Params& p, int64_t qt) {
   if (p.mode == kModeDense) return static_cast<int>((p.Lk + kBN - 1) / kBN);
   const int64_t r0 = qt * kBM;
   if (p.mode == kModeFilter) {
-    const int64_t last = min(r0 + kBM, p.Lq) - 1;
+    const int64_t last = p.q0 + min(r0 + kBM, p.Lq) - 1;   // position of the tile's last row
     return static_cast<int>(last / kBN + 1);
   }
-  if (r0 + kBM <= p.cap) return 0;  // every row of the tile keeps all its keys
-  return static_cast<int>(min64(sample_span(qt), kSampTilesMax));
+  if (p.q0 + r0 + kBM <= p.cap) return 0;  // every row of the tile keeps all its keys
+  return static_cast<int>(min64(sample_span(p.q0 + r0), kSampTilesMax));
 }
 
 __device__ __forceinline__ int item_ktile(const Params& p, int64_t qt, int j, int nt) {
   if (p.mode != kModeSample) return j;
-  return static_cast<int>((static_cast<int64_t>(j) * sample_span(qt)) / nt);
+  return static_cast<int>((static_cast<int64_t>(j) * sample_span(p.q0 + qt * kBM)) / nt);
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
@@ -147,12 +148,12 @@ __device__ __forceinline__ uint32_t sample_key16(uint32_t acc_bits) {
 constexpr int kMiniRows = 8;                       // rows per sampled mini-tile
 constexpr int kMinisPerTile = kBN / kMiniRows;     // 32
 
-// First key of mini-tile i (0 .. nt*32-1) of query tile qt: the mini-tiles
-// are spread evenly over the keys below the band [r0 - 128, r0 + 128), so
-// every region of the prefix is represented (a stratified sample), and each
-// stays inside it.
-__device__ __forceinline__ int mini_tile_row(int64_t qt, int i, int nt) {
-  const uint64_t span = static_cast<uint64_t>(qt * kBM - 128);     // keys [0, span)
+// First key of mini-tile i (0 .. nt*32-1) of the query tile whose first row
+// sits at position r0: the mini-tiles are spread evenly over the keys below
+// the band [r0 - 128, r0 + 128), so every region of the prefix is
+// represented (a stratified sample), and each stays inside it.
+__device__ __forceinline__ int mini_tile_row(int64_t r0, int i, int nt) {
+  const uint64_t span = static_cast<uint64_t>(r0 - 128);           // keys [0, span)
   const uint64_t nmini = static_cast<uint64_t>(nt) * kMinisPerTile;
   const uint64_t room = span - kMiniRows;                          // span >= 256 * nt
   return static_cast<int>((static_cast<uint64_t>(i) * room) / (nmini - 1 > 0 ? nmini - 1 : 1));
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (all 32-byte slices) into rows 8*lane .. 8*lane+7 of the stage.
             if (lane == 0) mbar_arrive_expect_tx(bar(FULL + s), stage_bytes);
             __syncwarp();
-            const int y = mini_tile_row(qt, j * kMinisPerTile + lane, nt);
+            const int y = mini_tile_row(p.q0 + qt * kBM, j * kMinisPerTile + lane, nt);
             for (int i = 0; i < p.sl.n; ++i)
               tma_load_2d(dst + p.sl.b_off[i] + lane * kMiniRows * p.sl.width[i], &maps.k8[p.sl.kind[i]],
                           p.sl.col[i] / ESIZE, y, bar(FULL + s));
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t pass = 0;
 #pragma unroll
               for (int q = 0; q < kChunk; ++q) pass |= (__uint_as_float(v[q]) >= tau ? 1u : 0u) << q;
-              const int64_t lim = t - s0;  // keys s0 .. t are causal
+              const int64_t lim = p.q0 + t - s0;  // keys s0 .. q0 + t are causal
               if (lim < kChunk - 1) pass &= lim < 0 ? 0u : ((2u << lim) - 1u);
               if (!row_ok) pass = 0;
               if (pass) {
@@ -491,24 +492,26 @@ __device__ __forceinline__ void warp_find_from_top(const unsigned int* hist, int
 // threshold; it is lowered to the smallest accumulator whose scaled score
 // equals that key's score, so the filter keeps whole ties.
 __global__ void __launch_bounds__(256) tau_kernel(const uint16_t* samp, int samp_ld, int64_t L,
-                                                  int cap, int target, float scale, float* tau) {
+                                                  int64_t q0, int cap, int target, float scale,
+                                                  float* tau) {
   __shared__ unsigned int hist_all[8][256];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + w;
-  if (t >= L) return;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + w;
+  if (row >= L) return;
+  const int64_t t = q0 + row;          // the query's key position
   unsigned int* hist = hist_all[w];
   if (t + 1 <= cap) {
-    if (lane == 0) tau[t] = -INFINITY;
+    if (lane == 0) tau[row] = -INFINITY;
     return;
   }
-  const int64_t qt = t / kBM;
-  const int ns = static_cast<int>(min64(sample_span(qt), kSampTilesMax));
+  const int64_t qt = row / kBM;
+  const int ns = static_cast<int>(min64(sample_span(q0 + qt * kBM), kSampTilesMax));
   if (ns == 0) {
-    if (lane == 0) tau[t] = -INFINITY;
+    if (lane == 0) tau[row] = -INFINITY;
     return;
   }
   const int n = ns * kBN;
-  const uint16_t* src = samp + t * samp_ld;
+  const uint16_t* src = samp + row * samp_ld;
   int R = static_cast<int>((static_cast<int64_t>(n) * target + t) / (t + 1));
   R = max(1, min(R, n));
   for (int i = lane; i < 256; i += 32) hist[i] = 0;
@@ -533,7 +536,7 @@ __global__ void __launch_bounds__(256) tau_kernel(const uint16_t* samp, int samp
     if (!(a > 0.0f) || !(sigma > 0.0f)) {
       // The sampled rank falls among ReLU zeros: keep every positive score
       // (smallest positive threshold) and let the select add zeros by index.
-      tau[t] = __uint_as_float(1u);
+      tau[row] = __uint_as_float(1u);
       return;
     }
     for (int i = 0; i < 64; ++i) {
@@ -543,7 +546,7 @@ __global__ void __launch_bounds__(256) tau_kernel(const uint16_t* samp, int samp
       else
         break;
     }
-    tau[t] = a;
+    tau[row] = a;
   }
 }
 
@@ -614,6 +617,7 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   p.k_idx = a.k_idx;
   p.Lq = a.Lq;
   p.Lk = a.Lk;
+  p.q0 = a.q0;
   p.nkb = nkb;
   p.stages = stages;
   p.off_b = a_bytes;
@@ -661,10 +665,10 @@ dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream) {
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-dsa_status launch_tau_select(const uint16_t* samp, int samp_ld, int64_t L, int cap, int target,
-                             float scale, float* tau, cudaStream_t stream) {
+dsa_status launch_tau_select(const uint16_t* samp, int samp_ld, int64_t L, int64_t q0, int cap,
+                             int target, float scale, float* tau, cudaStream_t stream) {
   const int64_t blocks = (L + 7) / 8;
-  tau_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(samp, samp_ld, L, cap, target,
+  tau_kernel<<<static_cast<unsigned int>(blocks), 256, 0, stream>>>(samp, samp_ld, L, q0, cap, target,
                                                                     scale, tau);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

@@ -25,6 +25,7 @@ struct IndexerLaunch {
   int esize;          // 1 = FP8 E4M3, 2 = BF16
   int d;              // index dim (elements)
   int64_t Lq, Lk;
+  int64_t q0;         // causal modes: query row i sits at key position q0 + i
   float scale;
   int mode;
   // filter
@@ -43,13 +44,15 @@ struct IndexerLaunch {
 dsa_status launch_indexer(const IndexerLaunch& a, cudaStream_t stream);
 
 // Threshold per query row from the sampled scores (raw accumulator domain).
-dsa_status launch_tau_select(const uint16_t* samp, int samp_ld, int64_t L, int cap, int target,
-                             float scale, float* tau, cudaStream_t stream);
+dsa_status launch_tau_select(const uint16_t* samp, int samp_ld, int64_t L, int64_t q0, int cap,
+                             int target, float scale, float* tau, cudaStream_t stream);
 
 // ---- select -------------------------------------------------------------------
 
 struct SelectLaunch {
-  int64_t L;
+  int64_t L;             // query rows
+  int64_t q0;            // query row t sits at key position q0 + t
+  int64_t Lk;            // key rows (q0 + L)
   int top_k;
   int cap;
   const unsigned long long* cand;
@@ -65,7 +68,7 @@ struct SelectLaunch {
   const void* k_idx;
   int esize, d;
   float scale;
-  unsigned long long* fb_scratch;  // [fb_ctas, L]
+  unsigned long long* fb_scratch;  // [fb_ctas, Lk]
   unsigned int* fb_hist;           // [fb_ctas, 4096]
   int* fb_slow;                    // [fb_ctas]
   int fb_ctas;                     // fallback rows handled by the grid-wide path
@@ -86,7 +89,7 @@ struct AttnLaunch {
   int H, D;
   float scale_log2;            // softmax scale * log2(e)
   int top_k;
-  // prefill: count(q) = min(top_k, q + 1), row base 0
+  // prefill: count(q) = min(top_k, q0 + q + 1), row base 0
   // decode:  count(q) = min(top_k, len_q), row base seq_start[q]
   const int64_t* seq_start;    // null for prefill
   int nsplit;                  // splits of the key list per query (1 = final output)
@@ -97,6 +100,7 @@ struct AttnLaunch {
   // is row (block_table[q * bt_ld + (s >> bs_log2)] << bs_log2) | (s & (2^bs_log2 - 1))
   const int32_t* block_table;
   int bt_ld, bs_log2;
+  int64_t q0;                  // prefill: query q sits at key position q0 + q (chunked prefill)
 };
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream);

@@ -270,7 +270,8 @@ __device__ void merge_by_index(const unsigned long long* a, int na, const unsign
 }
 
 struct SelParams {
-  int64_t L;
+  int64_t L;       // query rows
+  int64_t q0;      // query row t sits at key position q0 + t
   int top_k, cap;
   float scale;
   const unsigned long long* cand;
@@ -405,7 +406,8 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
   static_assert(kCandParts == 2 || kCandParts == 4, "two or four candidate lists per row");
   unsigned long long* lists = kCandParts == 4 ? sm.raw : sm.tmp;
   for (int64_t t = blockIdx.x; t < p.L; t += gridDim.x) {
-    const int m = static_cast<int>(min64(p.top_k, t + 1));
+    const int64_t qpos = p.q0 + t;   // the query's key position: keys 0 .. qpos are causal
+    const int m = static_cast<int>(min64(p.top_k, qpos + 1));
     int nl[kCandParts];
     int n = 0;
     bool overflow = false;
@@ -505,13 +507,14 @@ __global__ void __launch_bounds__(kSortThreads, 2) select_kernel(const SelParams
       __syncthreads();
       st = stats_read(sm.misc);
     }
-    sort_emit(sm, n, m, zero_mode, t, p.top_k, p.indices + t * p.top_k, st);
+    sort_emit(sm, n, m, zero_mode, qpos, p.top_k, p.indices + t * p.top_k, st);
     __syncthreads();
   }
 }
 
 struct FbParams {
-  int64_t L;
+  int64_t L;                     // key rows (stride of the scratch rows)
+  int64_t q0;                    // query row t sits at key position q0 + t
   int top_k;
   const void* q_idx;
   const void* k_idx;
@@ -600,9 +603,10 @@ __global__ void __launch_bounds__(kSelThreads) fb_score_kernel(const FbParams p)
   for (int64_t item = blockIdx.x; item < items; item += gridDim.x) {
     const int f = static_cast<int>(item / cpr), c = static_cast<int>(item % cpr);
     const int64_t t = p.fb_rows[f];
+    const int64_t pos = p.q0 + t;   // keys 0 .. pos are causal
     const int64_t s0 = static_cast<int64_t>(c) * kFbChunk;
-    if (s0 > t) continue;
-    const int64_t s1 = min64(t + 1, s0 + kFbChunk);
+    if (s0 > pos) continue;
+    const int64_t s1 = min64(pos + 1, s0 + kFbChunk);
     load_row_f32<ESIZE>(p.q_idx, t, p.d, qf);
     for (int i = threadIdx.x; i < kFbBins; i += blockDim.x) h[i] = 0u;
     __syncthreads();
@@ -645,7 +649,7 @@ __global__ void __launch_bounds__(kSortThreads, 1) fb_select_kernel(const FbPara
   static_assert(kPer * kSortThreads == kFbBins, "bins per thread");
   for (int f = blockIdx.x; f < nf; f += gridDim.x) {
     const int64_t t = p.fb_rows[f];
-    const int n = static_cast<int>(t + 1);
+    const int n = static_cast<int>(p.q0 + t + 1);
     const int m = min(p.top_k, n);
     const unsigned int* gh = p.hist + static_cast<int64_t>(f) * kFbBins;
     // thread i owns bins kFbBins-1-kPer*i .. kFbBins-kPer*(i+1) (descending)
@@ -726,7 +730,7 @@ __global__ void __launch_bounds__(kSortThreads, 1) fb_select_kernel(const FbPara
     }
     stats_reduce(slo, shi, sor, spos, misc);
     __syncthreads();
-    sort_emit(sm, static_cast<int>(total), m, false, t, p.top_k, p.indices + t * p.top_k,
+    sort_emit(sm, static_cast<int>(total), m, false, p.q0 + t, p.top_k, p.indices + t * p.top_k,
               stats_read(misc));
     __syncthreads();
   }
@@ -749,7 +753,7 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
   for (int w = blockIdx.x; w < nslow + extra; w += gridDim.x) {
     const int f = w < nslow ? p.slow[w] : p.slots + (w - nslow);
     const int64_t t = p.fb_rows[f];
-    const int n = static_cast<int>(t + 1);
+    const int n = static_cast<int>(p.q0 + t + 1);
     const int m = min(p.top_k, n);
     load_row_f32<ESIZE>(p.q_idx, t, p.d, qf);
     __syncthreads();
@@ -768,8 +772,8 @@ __global__ void __launch_bounds__(kSelThreads) fallback_kernel(const FbParams p)
 
 dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   const int P = 1 << (32 - __builtin_clz(std::max(a.top_k, 2) - 1));
-  SelParams p{a.L,      a.top_k,   a.cap,     a.scale,    a.cand,
-              a.cand_n, a.tau,     a.indices, a.fb_rows,  a.counters, a.force_fb_period};
+  SelParams p{a.L,      a.q0,    a.top_k,   a.cap,     a.scale,    a.cand,
+              a.cand_n, a.tau,   a.indices, a.fb_rows,  a.counters, a.force_fb_period};
   cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSelSmemBytes));
   if (e != cudaSuccess) return DSA_ERR_CUDA;
@@ -783,7 +787,7 @@ dsa_status launch_select(const SelectLaunch& a, cudaStream_t stream) {
   if (cudaMemsetAsync(a.fb_hist, 0, static_cast<size_t>(a.fb_ctas) * kFbBins * sizeof(unsigned int),
                       stream) != cudaSuccess)
     return DSA_ERR_CUDA;
-  FbParams f{a.L,       a.top_k,      a.q_idx,   a.k_idx,   a.esize,  a.d,     a.scale,
+  FbParams f{a.Lk,      a.q0,         a.top_k,   a.q_idx,   a.k_idx,  a.esize, a.d,     a.scale,
              a.fb_rows, a.counters,   a.indices, a.fb_scratch, a.fb_hist, a.fb_slow, a.fb_ctas};
   if (a.esize == 1)
     fb_score_kernel<1><<<4 * num_sms(), kSelThreads, 0, stream>>>(f);

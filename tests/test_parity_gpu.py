@@ -258,6 +258,61 @@ def test_prefill_workload_4k_all_rows(dsa):
     compare(x, w.idx_dtype, w.top_k, idx, O)
 
 
+# ------------------------------------------------------------------ prefill of a chunk of rows
+
+def run_chunk(dsa, x, q0, top_k, **kw):
+    """Rows q0 .. Lk-1 of x against keys 0 .. Lk-1 through dsa_prefill_chunk."""
+    Lk = x["q_idx"].shape[0]
+    q, k = to_dev(x["q_idx"][q0:]), to_dev(x["k_idx"])
+    if q.dtype == torch.uint16:
+        q, k = q.view(torch.bfloat16), k.view(torch.bfloat16)
+    idx, O = dsa.dsa_prefill_chunk(q, k, bf16(x["Q"][q0:]), bf16(x["K"]), bf16(x["V"]), top_k, **kw)
+    assert dsa.dsa_sync_status() == 0
+    return idx.cpu().numpy(), O.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("Lk,q0,top_k,H,D,d,idx_dtype", [
+    (2333, 1633, 256, 16, 128, 96, "fp8"),     # chunk start off every tile boundary
+    (5000, 4999, 2048, 16, 128, 128, "fp8"),   # one new token (decode as a chunk)
+    (3000, 64, 300, 4, 64, 160, "bf16"),       # most rows of the sequence, head dim 64
+    (4100, 2048, 1024, 3, 128, 128, "fp8"),    # chunk starting on a key-tile boundary
+])
+def test_prefill_chunk_matches_oracle_rows(dsa, Lk, q0, top_k, H, D, d, idx_dtype):
+    x = small_inputs(Lk, d, H, D, idx_dtype=idx_dtype, seed=21)
+    idx, O = run_chunk(dsa, x, q0, top_k)
+    rows = np.arange(q0, Lk, dtype=np.int64)
+    ri, ro = oracle.prefill_rows(x, idx_dtype, top_k, rows=rows)
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_prefill_chunk_forced_fallback(dsa, force_fallback):
+    x = small_inputs(6000, 128, 16, 128, seed=22)
+    force_fallback(9)
+    idx, O = run_chunk(dsa, x, 3500, 2048)
+    ri, ro = oracle.prefill_rows(x, "fp8", 2048, rows=np.arange(3500, 6000, dtype=np.int64))
+    assert np.array_equal(idx, ri)
+    assert np.abs(bits_to_f32(O) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_prefill_chunks_in_zigzag_order_equal_the_whole_prefill(dsa):
+    """The 32K workload split as for 4 ranks (8 zig-zag chunks): every chunk
+    through dsa_prefill_chunk against its key prefix gives, row for row, the
+    indices and outputs of the whole-sequence call."""
+    from sparse_attention_10_b200.zigzag import zigzag_chunks
+    w = synth.WORKLOADS["prefill_32k"]
+    x = synth.prefill_inputs_torch(w, device="cuda")
+    idx_all, O_all = dsa.dsa_prefill(x["q_idx"], x["k_idx"], x["Q"], x["K"], x["V"], w.top_k)
+    assert dsa.dsa_sync_status() == 0
+    for r in range(4):
+        for a, b in zigzag_chunks(w.L, 4, r):
+            idx, O = dsa.dsa_prefill_chunk(x["q_idx"][a:b], x["k_idx"][:b], x["Q"][a:b], x["K"][:b],
+                                           x["V"][:b], w.top_k)
+            assert dsa.dsa_sync_status() == 0
+            assert torch.equal(idx, idx_all[a:b]), (a, b)
+            assert torch.equal(O.view(torch.int16), O_all[a:b].view(torch.int16)), (a, b)
+
+
 # ------------------------------------------------------------------ prefill, full size
 
 def sampled_rows(L, k, n=2048, seed=0):
