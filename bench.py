@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the 4K/32K/64K prefill sub-lines")
+    ap.add_argument("--no-zigzag", action="store_true", help="skip the row-split (strong scaling) sub-line")
+    ap.add_argument("--no-fp8-path", action="store_true", help="skip the FP8 copy of BF16 index inputs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU-baseline sample time")
     ap.add_argument("--workload", default=PREFILL,
                     choices=["prefill_4k", "prefill_32k", "prefill_64k", "prefill_128k", "prefill_32k_bf16"],
@@ -555,6 +557,105 @@ def main():
                               "summary in profiles/ whose recorded source hash matches this kernel's source "
                               "(null when it does not)")
 
+    # --- the same sequence split over the ranks by query rows (zig-zag chunks, one all-gather
+    # of the key rows, dsa_prefill_chunk per chunk): strong scaling of one sequence
+    zz = None
+    if not args.no_zigzag:
+        from sparse_attention_10_b200.zigzag import prefill_sharded, zigzag_chunks
+        xs = x if seed == synth.SEED else synth.prefill_inputs_torch(w, seed=synth.SEED, device=dev)
+        chunks = zigzag_chunks(w.L, world, rank)
+        parts = {n_: [xs[n_][a_:b_].contiguous() for a_, b_ in chunks] for n_ in ("q_idx", "k_idx", "Q", "K", "V")}
+        ws_z = [torch.empty(dsa.dsa_prefill_chunk_workspace_size(b_ - a_, b_, w.d_idx, idt, w.H, w.D, w.top_k),
+                            dtype=torch.uint8, device=dev) for a_, b_ in chunks]
+        wsq = iter(())
+
+        def zchunk(qi, kf, Qi, Kf, Vf, top_k):
+            return dsa.dsa_prefill_chunk(qi, kf, Qi, Kf, Vf, top_k, workspace=next(wsq), stream=stream)
+
+        def zstep():
+            nonlocal wsq
+            wsq = iter(ws_z)
+            return prefill_sharded(parts["q_idx"], parts["k_idx"], parts["Q"], parts["K"], parts["V"], w.L,
+                                   w.top_k, world, rank, chunk_fn=zchunk)
+
+        for _ in range(max(1, args.warmup)):
+            zstep()
+        torch.cuda.synchronize()
+        nz = max(3, args.steps // 2)
+        barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(nz):
+            zstep()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        zms = max_over_ranks(e0.elapsed_time(e1)) / nz
+        if dsa.dsa_sync_status(stream) != 0:
+            raise RuntimeError("device-side error in the row-split prefill")
+        zz = {"value": w.L / (zms / 1000.0), "unit": "queries/s", "ms_per_step": zms, "scaling": "strong",
+              "chunks_of_rank0": zigzag_chunks(w.L, world, 0),
+              "how": f"one {w.name} sequence split over {world} rank(s) by query rows: 2 x {world} zig-zag "
+                     f"chunks, all-gather of k_idx/K/V rows (NCCL), dsa_prefill_chunk per chunk; the timed "
+                     f"region covers the all-gather and both chunks of every rank (max over ranks)"}
+        del parts, ws_z
+        if xs is not x:
+            del xs
+        torch.cuda.empty_cache()
+
+    # --- BF16 index inputs that are exact in FP8 E4M3 (the workload's small integers): the
+    # E4M3 copy runs the indexer on the FP8 tensor-core path with identical scores.  Each
+    # timed step converts both index tensors (dsa_index_to_fp8) and runs dsa_prefill on the copy.
+    fp8_path = None
+    if w.idx_dtype == "bf16" and not args.no_fp8_path:
+        q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+        bad = torch.empty(2, dtype=torch.int64, device=dev)
+        dsa.dsa_index_to_fp8(q, out=q8, inexact=bad[0:1], stream=stream)
+        dsa.dsa_index_to_fp8(k, out=k8, inexact=bad[1:2], stream=stream)
+        torch.cuda.synchronize()
+        if int(bad.sum().item()) == 0:
+            ws8 = torch.empty(dsa.dsa_prefill_workspace_size(w.L, w.d_idx, dsa.IDX_FP8_E4M3, w.H, w.D, w.top_k),
+                              dtype=torch.uint8, device=dev)
+            idx8 = torch.empty_like(idx)
+            O8 = torch.empty_like(O)
+
+            def step8():
+                dsa.dsa_index_to_fp8(q, out=q8, inexact=bad[0:1], stream=stream)
+                dsa.dsa_index_to_fp8(k, out=k8, inexact=bad[1:2], stream=stream)
+                dsa.dsa_prefill(q8, k8, Q, K, V, w.top_k, indices=idx8, O=O8, workspace=ws8, stream=stream)
+
+            for _ in range(args.warmup):
+                step8()
+            torch.cuda.synchronize()
+            barrier()
+            e0.record(stream)
+            for _ in range(args.steps):
+                step8()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            ms8 = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+            dsa.dsa_stage_timing(True)
+            for _ in range(args.steps):
+                step8()
+            torch.cuda.synchronize()
+            dsa.dsa_stage_timing(False)
+            st8 = {k_: v[0] / args.steps for k_, v in dsa.dsa_stage_times().items() if v[1] > 0}
+            if dsa.dsa_sync_status(stream) != 0:
+                raise RuntimeError("device-side error on the FP8 index path")
+            same = bool(torch.equal(idx8, idx) and torch.equal(O8.view(torch.int16), O.view(torch.int16)))
+            t8 = work["indexer_flops"] / (st8["indexer_filter"] / 1000.0) / 1e12
+            fp8_path = {"value": world * w.L / (ms8 / 1000.0), "unit": "queries/s", "ms_per_step": ms8,
+                        "stage_ms": st8, "matches_bf16_call": same,
+                        "indexer": {"tflops": t8, "dtype": "fp8", "peak": fp8_peak, "frac": t8 / fp8_peak,
+                                    "peak_source": "FP8 measured in this run"},
+                        "how": "per step: dsa_index_to_fp8 on q_idx and k_idx (inside the timed region), "
+                               "then dsa_prefill with the E4M3 copies"}
+            del ws8, idx8, O8
+        del q8, k8, bad
+        torch.cuda.empty_cache()
+
     # --- end to end through the public API with host buffers.  A serving loop
     # pipelines the transfers: while step i computes, step i+1's inputs go up
     # and step i-1's outputs come down (one stream each, double-buffered device
@@ -735,7 +836,7 @@ def main():
             "config": line_config(w, world),
             "indexer_tflops": indexer_tflops, "gather_gbs": gather_gbs, "indexer": indexer,
             "attention": attention, "stage_ms": st_ms, "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "peaks_in_run": run_peaks, "configs": configs,
+            "peaks_in_run": run_peaks, "configs": configs, "row_split": zz, "fp8_index_path": fp8_path,
             "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": clocks.summary(),
             "decode": decode, "select_stats": stats,
         }

@@ -263,6 +263,24 @@ dsa_status dsa_debug_wait_timeout(uint64_t limit_ns, void* stream);
 dsa_status dsa_debug_force_fallback(int period);
 
 /*
+ * dsa_index_to_fp8 — lossless FP8 copy of BF16 indexer inputs.  Section 7.2
+ * of the page runs the 128K indexer in BF16 and section 4.1 the index stage
+ * in FP8; when every BF16 value is exactly an FP8 E4M3 value (small integers,
+ * for instance), the E4M3 copy gives bit-identical indexer scores, so
+ * dsa_prefill can take it (idx_dtype FP8) and run the indexer on the FP8
+ * tensor-core path.  Writes out_fp8[i] = E4M3(in_bf16[i]) (round to nearest,
+ * saturating) and counts in *inexact the values whose copy differs from the
+ * input (NaN included).  Use the copy only when *inexact == 0 (read it after
+ * synchronising the stream); the count is reset by the call.
+ *   in_bf16  device [n] BF16, 16-byte aligned
+ *   out_fp8  device [n] bytes, 8-byte aligned, written
+ *   inexact  device uint64, written
+ * n must be a positive multiple of 8 (any index dim of 16 or more does).
+ */
+dsa_status dsa_index_to_fp8(const void* in_bf16, int64_t n, void* out_fp8, uint64_t* inexact,
+                            void* stream);
+
+/*
  * dsa_gather_probe — diagnostic: the memory ceiling of the attention's
  * gather.  The attention of section 3.3 reads, for each query, the K and V
  * rows of its kept keys (section 4.2: one K/V shared by every head), random

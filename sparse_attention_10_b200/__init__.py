@@ -20,7 +20,7 @@ __all__ = [
     "dsa_sync_status", "dsa_last_stats", "dsa_debug_wait_timeout", "dsa_debug_force_fallback", "IDX_FP8_E4M3", "IDX_BF16",
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
     "dsa_decode_paged_workspace_size", "dsa_decode_paged", "dsa_gather_probe",
-    "dsa_prefill_chunk_workspace_size", "dsa_prefill_chunk",
+    "dsa_prefill_chunk_workspace_size", "dsa_prefill_chunk", "dsa_index_to_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -66,6 +66,7 @@ def load() -> ctypes.CDLL:
         "dsa_decode_paged": ([P, P, P, I64, I, P, I, P, I, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ,
                               P], I),
         "dsa_gather_probe": ([P, I64, I, P, P, I, I, I, P, P], I),
+        "dsa_index_to_fp8": ([P, I64, P, P, P], I),
         "dsa_stage_timing": ([I], I),
         "dsa_stage_times": ([ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64), I], I),
     }
@@ -305,6 +306,21 @@ def dsa_gather_probe(indices: torch.Tensor, K: torch.Tensor, V: torch.Tensor, ct
     _check(load().dsa_gather_probe(_dev(indices, "indices"), L, top_k, _dev(K, "K"), _dev(V, "V"), D,
                                    int(ctas_per_sm), int(stages), _dev(sink, "sink"), _stream(stream)),
            "dsa_gather_probe")
+
+
+def dsa_index_to_fp8(x: torch.Tensor, out: Optional[torch.Tensor] = None,
+                     inexact: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """E4M3 copy of a BF16 index tensor -> (copy as uint8, device count of values it changed).
+    The copy gives the same indexer scores only when the count is zero."""
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bfloat16")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if inexact is None:
+        inexact = torch.empty(1, dtype=torch.int64, device=x.device)
+    _check(load().dsa_index_to_fp8(_dev(x, "x"), x.numel(), _dev(out, "out"), _dev(inexact, "inexact"),
+                                   _stream(stream)), "dsa_index_to_fp8")
+    return out, inexact
 
 
 def dsa_sync_status(stream=None) -> int:

@@ -258,6 +258,42 @@ def test_prefill_workload_4k_all_rows(dsa):
     compare(x, w.idx_dtype, w.top_k, idx, O)
 
 
+# ------------------------------------------------------------------ FP8 copy of BF16 index inputs
+
+def test_index_to_fp8_is_exact_on_integers_and_counts_the_rest(dsa):
+    v = torch.tensor([0, 1, -1, 2, -3, 4, 0.5, 448, -448, 0.1, 3.3, 1000, float("nan"), -0.0, 17, 2 ** -9],
+                     dtype=torch.bfloat16, device="cuda")
+    out, bad = dsa.dsa_index_to_fp8(v)
+    torch.cuda.synchronize()
+    back = out.view(torch.float8_e4m3fn).float()
+    exact = (back == v.float())
+    # 0.1, 3.3, 1000 (beyond 448), NaN and 17 (needs 4 mantissa bits) do not survive
+    assert int(bad.item()) == 5
+    assert exact[:9].all() and exact[13] and exact[15]
+    ref = v.float().to(torch.float8_e4m3fn).view(torch.uint8)
+    fin = torch.isfinite(v.float()) & (v.float().abs() <= 448)
+    assert torch.equal(out[fin], ref[fin])
+
+
+def test_prefill_on_the_fp8_copy_of_bf16_integer_inputs_is_identical(dsa):
+    """The 128K workload's settings (BF16 index dim 160, top_k 2048) at L = 9000:
+    the E4M3 copy of the integer inputs runs the FP8 indexer and gives the same
+    indices and outputs as the BF16 call, and the oracle's."""
+    x = small_inputs(9000, 160, 16, 128, idx_dtype="bf16", seed=23)
+    q, k = bf16(x["q_idx"]), bf16(x["k_idx"])
+    q8, bq = dsa.dsa_index_to_fp8(q)
+    k8, bk = dsa.dsa_index_to_fp8(k)
+    assert int(bq.item()) == 0 and int(bk.item()) == 0
+    Q, K, V = bf16(x["Q"]), bf16(x["K"]), bf16(x["V"])
+    i16, o16 = dsa.dsa_prefill(q, k, Q, K, V, 2048)
+    i8, o8 = dsa.dsa_prefill(q8, k8, Q, K, V, 2048)
+    assert dsa.dsa_sync_status() == 0
+    assert torch.equal(i8, i16)
+    assert torch.equal(o8.view(torch.int16), o16.view(torch.int16))
+    rows = np.unique(np.concatenate([np.arange(0, 9000, 211), [2047, 2048, 8999]])).astype(np.int64)
+    compare(x, "bf16", 2048, i8.cpu().numpy(), o8.view(torch.int16).cpu().numpy().view(np.uint16), rows=rows)
+
+
 # ------------------------------------------------------------------ prefill of a chunk of rows
 
 def run_chunk(dsa, x, q0, top_k, **kw):
