@@ -396,8 +396,8 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   unsigned long long* bufB = bufA + kSmemKeys;                     // [kSmemKeys]
   uint32_t* cnt = reinterpret_cast<uint32_t*>(bufB + kSmemKeys);   // [warps][256]
   uint32_t* dbase = cnt + kSelWarps * 256;                         // [256]
-  uint32_t* wsum = dbase + 256;                                    // [warps]
-  int* sh = reinterpret_cast<int*>(wsum + kSelWarps);              // [8]
+  uint32_t* wsum = dbase + 256;                                    // [2][warps]
+  int* sh = reinterpret_cast<int*>(wsum + 2 * kSelWarps);          // [8]
   unsigned int* h256 = dbase;                                      // fallback path histogram
   if (*p.invalid) return;
   const int b = blockIdx.x;
@@ -409,57 +409,83 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   const unsigned int* hist = p.hist + static_cast<int64_t>(b) * kHistBins;
   int32_t* out = p.indices + static_cast<int64_t>(b) * p.top_k;
 
-  // Bin of the m-th best score (bins scanned from the top by warp 0).  Bin 0
-  // (score +0) is not counted by the scan: every key not in a higher bin.
-  if (threadIdx.x < 32) {
-    unsigned int local = 0;
-    for (int i = 0; i < kHistBins / 32; ++i) {
-      const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
-      if (bb > 0) local += hist[bb];
+  // Bin of the m-th best score.  The histogram is staged in shared memory
+  // (bufB is free until the sort); thread i owns bins 2047 - 2i and 2046 - 2i,
+  // a block-wide prefix from the top finds the bin.  Bin 0 (score +0) is not
+  // counted by the scan: it holds every key not counted in a higher bin.
+  {
+    unsigned int* hs = reinterpret_cast<unsigned int*>(bufB);
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hs[i] = i > 0 ? hist[i] : 0u;
+    if (threadIdx.x == 0) {
+      sh[3] = 0;            // OR of score words
+      sh[4] = -1;           // AND of score words
     }
-    const unsigned int above0 = __reduce_add_sync(0xFFFFFFFFu, local);
-    if (lane == 31) local += static_cast<unsigned int>(n) - above0;
+    __syncthreads();
+    constexpr int kBinsPer = kHistBins / kSelThreads;
+    unsigned int loc[kBinsPer], local = 0;
+#pragma unroll
+    for (int q = 0; q < kBinsPer; ++q) {
+      loc[q] = hs[kHistBins - 1 - kBinsPer * threadIdx.x - q];
+      local += loc[q];
+    }
     unsigned int incl = local;
+#pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const unsigned int y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
       if (lane >= o) incl += y;
     }
-    const unsigned int ballot = __ballot_sync(0xFFFFFFFFu, incl >= static_cast<unsigned int>(m));
-    const int src = __ffs(ballot) - 1;
-    if (lane == src) {
-      unsigned int run = incl - local;
-      for (int i = 0; i < kHistBins / 32; ++i) {
-        const int bb = kHistBins - 1 - (kHistBins / 32) * lane - i;
-        run += bb > 0 ? hist[bb] : static_cast<unsigned int>(n) - above0;
-        if (run >= static_cast<unsigned int>(m)) {
-          sh[0] = bb;
-          sh[1] = static_cast<int>(run);  // keys in bins >= bb
-          break;
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    unsigned int before = 0, above0 = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      const unsigned int x = wsum[w];
+      before += w < warp ? x : 0u;
+      above0 += x;
+    }
+    unsigned int run = before + incl - local;
+    if (threadIdx.x == kSelThreads - 1) {        // its last bin is bin 0
+      loc[kBinsPer - 1] = static_cast<unsigned int>(n) - above0;
+      local += loc[kBinsPer - 1];
+    }
+    if (run < static_cast<unsigned int>(m) && run + local >= static_cast<unsigned int>(m)) {
+#pragma unroll
+      for (int q = 0; q < kBinsPer; ++q) {
+        if (run < static_cast<unsigned int>(m) && run + loc[q] >= static_cast<unsigned int>(m)) {
+          sh[0] = kHistBins - 1 - kBinsPer * threadIdx.x - q;
+          sh[1] = static_cast<int>(run + loc[q]);  // keys in bins >= that bin
         }
+        run += loc[q];
       }
     }
-    if (lane == 0) {
-      sh[2] = 0;            // compacted so far
-      sh[3] = 0;            // OR of score words
-      sh[4] = -1;           // AND of score words
-    }
+    __syncthreads();
   }
-  __syncthreads();
   const uint32_t bin = static_cast<uint32_t>(sh[0]);
   const int ncand = sh[1];
 
   if (ncand <= kSmemKeys) {
     // Stable compaction of the candidates (score bin >= bin) in index order.
+    // Eight consecutive scores per thread and round; the next round's scores
+    // are loaded before this round's block scan, and the per-warp counts
+    // alternate between two arrays, so a round needs one barrier.
     uint32_t o_or = 0u, o_and = 0xFFFFFFFFu;
-    // eight consecutive scores per thread and round: the loads of a round
-    // are independent, so the rounds (each a block scan) are few
     constexpr int kPer = 8;
-    for (int s0 = 0; s0 < n; s0 += kSelThreads * kPer) {
-      const int s = s0 + threadIdx.x * kPer;
-      float v[kPer];
-      uint32_t flags = 0;
+    constexpr int kRound = kSelThreads * kPer;
+    const int rounds = (n + kRound - 1) / kRound;
+    float vn[kPer];
+    auto load = [&](int r) {
+      const int s = r * kRound + threadIdx.x * kPer;
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) v[k] = s + k < n ? sc[s + k] : 0.0f;
+      for (int k = 0; k < kPer; ++k) vn[k] = s + k < n ? sc[s + k] : 0.0f;
+    };
+    load(0);
+    uint32_t done = 0;
+    for (int r = 0; r < rounds; ++r) {
+      float v[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) v[k] = vn[k];
+      if (r + 1 < rounds) load(r + 1);
+      const int s = r * kRound + threadIdx.x * kPer;
+      uint32_t flags = 0;
 #pragma unroll
       for (int k = 0; k < kPer; ++k)
         if (s + k < n && (__float_as_uint(v[k]) >> 20) >= bin) flags |= 1u << k;
@@ -470,35 +496,32 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
         const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (lane == 31) wsum[warp] = incl;
+      uint32_t* ws = wsum + (r & 1) * kSelWarps;
+      if (lane == 31) ws[warp] = incl;
       __syncthreads();
-      if (warp == 0) {
-        const uint32_t x = wsum[lane];
-        uint32_t wi = x;
+      const uint32_t x = ws[lane];
+      uint32_t wi = x;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
-          if (lane >= o) wi += y;
-        }
-        wsum[lane] = wi - x;        // exclusive warp offsets
-        if (lane == 31) sh[5] = static_cast<int>(wi);
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, wi, o);
+        if (lane >= o) wi += y;
       }
-      __syncthreads();
-      int pos = sh[2] + static_cast<int>(wsum[warp] + incl - c);
+      const uint32_t woff = __shfl_sync(0xFFFFFFFFu, wi - x, warp);
+      const uint32_t total = __shfl_sync(0xFFFFFFFFu, wi, 31);
+      uint32_t pos = done + woff + incl - c;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) {
         if (flags & (1u << k)) {
           const uint32_t bits = __float_as_uint(v[k]);
           o_or |= bits;
           o_and &= bits;
-          if (pos < kSmemKeys) bufA[pos] = score_key(v[k], static_cast<uint32_t>(s + k));
+          if (pos < static_cast<uint32_t>(kSmemKeys)) bufA[pos] = score_key(v[k], static_cast<uint32_t>(s + k));
           ++pos;
         }
       }
-      __syncthreads();
-      if (threadIdx.x == 0) sh[2] += sh[5];
-      __syncthreads();
+      done += total;
     }
+    if (threadIdx.x == 0) sh[2] = static_cast<int>(done);
     o_or = __reduce_or_sync(0xFFFFFFFFu, o_or);
     o_and = __reduce_and_sync(0xFFFFFFFFu, o_and);
     if (lane == 0) {
@@ -591,7 +614,7 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
 
   DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid};
   const size_t smem = static_cast<size_t>(2 * kSmemKeys) * 8 +
-                      (kSelWarps * 256 + 256 + kSelWarps + 8) * 4;
+                      (kSelWarps * 256 + 256 + 2 * kSelWarps + 8) * 4;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
