@@ -210,6 +210,49 @@ dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int
                             float idx_scale, float attn_scale, void* O, int32_t* indices,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace dsa_decode_multi needs (T new tokens per sequence). */
+size_t dsa_decode_multi_workspace_size(int B, int T, int64_t total_rows, int d_idx, int idx_dtype,
+                                       int H, int D, int top_k);
+
+/*
+ * dsa_decode_multi — dsa_decode with T new tokens per sequence (1 <= T <= 4):
+ * speculative drafts, or a short chunk of prompt appended to each sequence.
+ * The T tokens' rows are the last T rows of each sequence in the cache; token
+ * j (0-based) of sequence b sits at position len_b - T + j and sees rows
+ * 0 .. len_b - T + j (causal among the new tokens too), as sections 3.2-3.3
+ * define for any query.  The index cache is read once for all T tokens.
+ *   q_idx    device [B, T, d_idx];  Q device [B, T, H, D] BF16
+ *   O        device [B, T, H, D] BF16, written
+ *   indices  device [B, T, top_k] int32, written when non-null (positions
+ *            within the sequence, -1 padded)
+ * Every other argument is that of dsa_decode; every length must be >= T.
+ * T > 1 needs index rows of 64, 128 or 256 bytes (FP8 d 64/128/256, BF16 d
+ * 64/128); other shapes return DSA_ERR_UNSUPPORTED.  T = 1 is dsa_decode.
+ */
+dsa_status dsa_decode_multi(const void* k_idx, const void* K, const void* V,
+                            const int64_t* seq_start, int B, int T, int64_t total_rows,
+                            int64_t max_len, int idx_dtype, int d_idx, int D, const void* q_idx,
+                            const void* Q, int H, int top_k, float idx_scale, float attn_scale,
+                            void* O, int32_t* indices, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/* Bytes of device workspace dsa_decode_paged_multi needs. */
+size_t dsa_decode_paged_multi_workspace_size(int B, int T, int64_t max_len, int d_idx,
+                                             int idx_dtype, int H, int D, int top_k);
+
+/*
+ * dsa_decode_paged_multi — dsa_decode_multi over a block-paged cache: the
+ * layout, block table and checks of dsa_decode_paged, T new tokens per
+ * sequence as in dsa_decode_multi (seq_lens[b] counts them; each >= T).
+ */
+dsa_status dsa_decode_paged_multi(const void* k_idx, const void* K, const void* V,
+                                  int64_t num_blocks, int block_size, const int32_t* block_table,
+                                  int max_blocks, const int32_t* seq_lens, int B, int T,
+                                  int64_t max_len, int idx_dtype, int d_idx, int D,
+                                  const void* q_idx, const void* Q, int H, int top_k,
+                                  float idx_scale, float attn_scale, void* O, int32_t* indices,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * dsa_sync_status — synchronise `stream`, then read and clear the current
  * device's status word (the first device-side error since the last read).

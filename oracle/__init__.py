@@ -151,6 +151,38 @@ def decode(inp: dict, idx_dtype: str, top_k: int, idx_scale=None, attn_scale=Non
     return indices, O
 
 
+def decode_multi(inp: dict, idx_dtype: str, top_k: int, idx_scale=None, attn_scale=None,
+                 want_o: bool = True, nthreads: int = 0):
+    """One decode step with T new tokens per sequence: indices [B, T, top_k], O [B, T, H, D].
+
+    inp holds the contiguous cache (k_idx, K, V, seq_start) and q_idx [B, T, d],
+    Q [B, T, H, D].  The new tokens are the last T rows of each sequence; token j
+    sits at position len_b - T + j and, as any query of the DeepSeek Sparse
+    Attention page (sections 3.2-3.3), sees the rows up to its own position.
+    Each token is an ordinary decode over its causal prefix of the sequence.
+    """
+    q_idx = np.asarray(inp["q_idx"])
+    B, T, d = q_idx.shape
+    ss = np.asarray(inp["seq_start"], dtype=np.int64)
+    rows, starts = [], [0]
+    for b in range(B):
+        n_b = int(ss[b + 1] - ss[b])
+        for j in range(T):
+            n = n_b - T + 1 + j
+            rows.append(np.arange(ss[b], ss[b] + n, dtype=np.int64))
+            starts.append(starts[-1] + n)
+    rows = np.concatenate(rows)
+    flat = {"k_idx": np.asarray(inp["k_idx"])[rows], "q_idx": q_idx.reshape(B * T, d),
+            "seq_start": np.asarray(starts, dtype=np.int64)}
+    if want_o:
+        Q = np.asarray(inp["Q"])
+        flat["K"] = np.asarray(inp["K"])[rows]
+        flat["V"] = np.asarray(inp["V"])[rows]
+        flat["Q"] = Q.reshape((B * T,) + Q.shape[2:])
+    idx, O = decode(flat, idx_dtype, top_k, idx_scale, attn_scale, want_o, nthreads)
+    return idx.reshape(B, T, top_k), (None if O is None else O.reshape((B, T) + O.shape[1:]))
+
+
 def decode_paged(inp: dict, idx_dtype: str, top_k: int, idx_scale=None, attn_scale=None,
                  want_o: bool = True, nthreads: int = 0):
     """One decode step over a block-paged cache: indices [B, top_k] and O [B, H, D].

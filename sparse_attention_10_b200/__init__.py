@@ -21,6 +21,8 @@ __all__ = [
     "LIB_PATH", "dsa_stage_timing", "dsa_stage_times", "STAGES", "dsa_decode_static",
     "dsa_decode_paged_workspace_size", "dsa_decode_paged", "dsa_gather_probe",
     "dsa_prefill_chunk_workspace_size", "dsa_prefill_chunk", "dsa_index_to_fp8",
+    "dsa_decode_multi_workspace_size", "dsa_decode_multi", "dsa_decode_paged_multi_workspace_size",
+    "dsa_decode_paged_multi",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsa.so")
@@ -56,6 +58,11 @@ def load() -> ctypes.CDLL:
         "dsa_prefill_chunk_workspace_size": ([I64, I64, I, I, I, I, I], SZ),
         "dsa_prefill_chunk": ([P, P, I, I, F, P, P, P, I64, I64, I, I, F, I, P, P, P, SZ, P], I),
         "dsa_decode_workspace_size": ([I, I64, I, I, I, I, I], SZ),
+        "dsa_decode_multi_workspace_size": ([I, I, I64, I, I, I, I, I], SZ),
+        "dsa_decode_multi": ([P, P, P, P, I, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ, P], I),
+        "dsa_decode_paged_multi_workspace_size": ([I, I, I64, I, I, I, I, I], SZ),
+        "dsa_decode_paged_multi": ([P, P, P, I64, I, P, I, P, I, I, I64, I, I, I, P, P, I, I, F, F, P, P, P,
+                                    SZ, P], I),
         "dsa_decode": ([P, P, P, P, I, I64, I64, I, I, I, P, P, I, I, F, F, P, P, P, SZ, P], I),
         "dsa_sync_status": ([P], I),
         "dsa_last_stats": ([P, ctypes.POINTER(ctypes.c_int64), P], I),
@@ -270,6 +277,77 @@ def dsa_decode_paged(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bloc
                               _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
                               _stream(stream))
     _check(st, "dsa_decode_paged")
+    return O, indices
+
+
+def dsa_decode_multi(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_start: torch.Tensor,
+                     q_idx: torch.Tensor, Q: torch.Tensor, top_k: int, max_len: int,
+                     idx_scale: Optional[float] = None, attn_scale: Optional[float] = None,
+                     O: Optional[torch.Tensor] = None, indices: Optional[torch.Tensor] = None,
+                     want_indices: bool = True, workspace: Optional[torch.Tensor] = None,
+                     stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """One decode step with T new tokens per sequence (q_idx [B, T, d], Q [B, T, H, D]) over a
+    ragged contiguous cache -> (O [B, T, H, D] bf16, indices [B, T, top_k] or None)."""
+    lib = load()
+    B, T, d = q_idx.shape
+    _, _, H, D = Q.shape
+    total = k_idx.shape[0]
+    idt = _idx_dtype(q_idx)
+    dev = q_idx.device
+    if O is None:
+        O = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    if indices is None and want_indices:
+        indices = torch.empty((B, T, top_k), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(int(lib.dsa_decode_multi_workspace_size(B, T, total, d, idt, H, D, top_k)),
+                                dtype=torch.uint8, device=dev)
+    if seq_start.dtype != torch.int64:
+        raise ValueError("seq_start must be int64")
+    st = lib.dsa_decode_multi(_dev(k_idx, "k_idx"), _dev(K, "K"), _dev(V, "V"), _dev(seq_start, "seq_start"),
+                              B, T, total, int(max_len), idt, d, D, _dev(q_idx, "q_idx"), _dev(Q, "Q"), H, top_k,
+                              _scale(idx_scale), _scale(attn_scale), _dev(O, "O"),
+                              _dev(indices, "indices") if indices is not None else None,
+                              _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _check(st, "dsa_decode_multi")
+    return O, indices
+
+
+def dsa_decode_paged_multi(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block_table: torch.Tensor,
+                           seq_lens: torch.Tensor, q_idx: torch.Tensor, Q: torch.Tensor, top_k: int,
+                           max_len: int, idx_scale: Optional[float] = None,
+                           attn_scale: Optional[float] = None, O: Optional[torch.Tensor] = None,
+                           indices: Optional[torch.Tensor] = None, want_indices: bool = True,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """dsa_decode_multi over a block-paged cache (layout of dsa_decode_paged)."""
+    lib = load()
+    B, T, d = q_idx.shape
+    _, _, H, D = Q.shape
+    num_blocks, block_size = k_idx.shape[0], k_idx.shape[1]
+    if block_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise ValueError("block_table and seq_lens must be int32")
+    if block_table.dim() != 2 or block_table.shape[0] != B or seq_lens.shape != (B,):
+        raise ValueError("block_table must be [B, max_blocks] and seq_lens [B]")
+    idt = _idx_dtype(q_idx)
+    dev = q_idx.device
+    if O is None:
+        O = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=dev)
+    if indices is None and want_indices:
+        indices = torch.empty((B, T, top_k), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(int(lib.dsa_decode_paged_multi_workspace_size(B, T, int(max_len), d, idt, H, D,
+                                                                              top_k)),
+                                dtype=torch.uint8, device=dev)
+    st = lib.dsa_decode_paged_multi(_dev(k_idx, "k_idx"), _dev(K, "K"), _dev(V, "V"), num_blocks, block_size,
+                                    _dev(block_table, "block_table"), block_table.shape[1],
+                                    _dev(seq_lens, "seq_lens"), B, T, int(max_len), idt, d, D,
+                                    _dev(q_idx, "q_idx"), _dev(Q, "Q"), H, top_k, _scale(idx_scale),
+                                    _scale(attn_scale), _dev(O, "O"),
+                                    _dev(indices, "indices") if indices is not None else None,
+                                    _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                                    _stream(stream))
+    _check(st, "dsa_decode_paged_multi")
     return O, indices
 
 

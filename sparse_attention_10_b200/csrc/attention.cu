@@ -89,6 +89,7 @@ struct AttnParams {
   const int32_t* block_table;   // paged decode cache, else null
   int bt_ld, bs_log2;
   int64_t q0;                   // prefill: query q sits at key position q0 + q
+  int qpt;                      // decode: queries per sequence
 };
 
 template <int D>
@@ -131,9 +132,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     const int sp = static_cast<int>(item % p.nsplit);
     int64_t row_base = 0;
     int count;
+    const int64_t sq = p.seq_start ? q / p.qpt : q;   // decode: the query's sequence
+    int64_t qlen = 0;                                   // decode: rows the query sees
     if (p.seq_start) {
-      row_base = p.seq_start[q];
-      count = static_cast<int>(min64(p.top_k, p.seq_start[q + 1] - row_base));
+      row_base = p.seq_start[sq];
+      qlen = p.seq_start[sq + 1] - row_base - (p.qpt - 1 - q % p.qpt);
+      count = static_cast<int>(min64(p.top_k, qlen));
     } else {
       count = static_cast<int>(min64(p.top_k, p.q0 + q + 1));
     }
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
     const int n = end - begin;
     const int32_t* ids = p.idx + q * p.ld_idx + begin;
     // rows a query may read: its causal prefix (prefill) or its sequence (decode)
-    const int row_limit = p.seq_start ? static_cast<int>(p.seq_start[q + 1] - row_base)
+    const int row_limit = p.seq_start ? static_cast<int>(qlen)
                                       : static_cast<int>(min64(p.q0 + q + 1, 0x7FFFFFFF));
     // a paged cache's key rows are absolute (translated below)
     const int64_t kv_base = p.block_table ? 0 : row_base;
@@ -165,7 +169,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
       const int s = sIds[i];
       int r = (s >= 0 && s < row_limit) ? s : -1;
       if (p.block_table && r >= 0)   // position in the sequence -> row of the block pool
-        r = (__ldg(p.block_table + q * p.bt_ld + (r >> p.bs_log2)) << p.bs_log2) |
+        r = (__ldg(p.block_table + sq * p.bt_ld + (r >> p.bs_log2)) << p.bs_log2) |
             (r & ((1 << p.bs_log2) - 1));
       sIds[i] = r;
     }
@@ -393,7 +397,7 @@ template <int D>
 dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   AttnParams p{a.Q,      a.K,    a.V,       a.idx,         a.ld_idx, a.nq,
                a.H,      a.scale_log2, a.top_k, a.seq_start, a.nsplit, a.O,
-               a.part,   a.invalid, a.block_table, a.bt_ld, a.bs_log2, a.q0};
+               a.part,   a.invalid, a.block_table, a.bt_ld, a.bs_log2, a.q0, std::max(a.qpt, 1)};
   const size_t smem = AttnSmem<D>::kBytes;
   static_assert(AttnSmem<D>::kStages * 2 * AttnSmem<D>::kTile >=
                     (4 * 16 * 2 + 4 * 16 * AttnSmem<D>::kMergeRow) * 4,

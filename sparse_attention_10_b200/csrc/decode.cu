@@ -85,13 +85,14 @@ __device__ __forceinline__ float dot_row(const float* q, const void* base, int64
   return acc[0];
 }
 
-// seq_start must start at 0, end at total_rows, and give lengths in [1, max_len].
+// seq_start must start at 0, end at total_rows, and give lengths in [nq, max_len]
+// (nq new tokens per sequence sit at its last nq rows).
 __global__ void validate_kernel(const int64_t* seq_start, int B, int64_t total_rows,
-                                int64_t max_len, int* invalid) {
+                                int64_t max_len, int nq, int* invalid) {
   bool bad = false;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int64_t len = seq_start[b + 1] - seq_start[b];
-    bad |= len < 1 || len > max_len;
+    bad |= len < nq || len > max_len;
   }
   if (threadIdx.x == 0) bad |= seq_start[0] != 0 || seq_start[B] != total_rows;
   if (__syncthreads_or(bad) && threadIdx.x == 0) {
@@ -104,7 +105,7 @@ __global__ void validate_kernel(const int64_t* seq_start, int B, int64_t total_r
 // every block a sequence reaches in [0, num_blocks).  CTA b also writes the
 // sum of the lengths before sequence b (and, for the last, the total), which
 // the later stages use as seq_start.
-__global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t max_len,
+__global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t max_len, int nq,
                                       const int32_t* table, int bt_ld, int bs_log2,
                                       int64_t num_blocks, int64_t* seq_start_out, int* invalid) {
   __shared__ long long wsum[32];
@@ -116,7 +117,7 @@ __global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t ma
   for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xFFFFFFFFu, before, o);
   if (lane == 0) wsum[warp] = before;
   const int64_t len = seq_lens[b];
-  bool bad = len < 1 || len > max_len || ((len - 1) >> bs_log2) >= bt_ld;
+  bool bad = len < nq || len > max_len || ((len - 1) >> bs_log2) >= bt_ld;
   if (!bad) {
     const int64_t nblk = ((len - 1) >> bs_log2) + 1;
     const int32_t* row = table + static_cast<int64_t>(b) * bt_ld;
@@ -140,16 +141,30 @@ __global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t ma
 
 struct ScanParams {
   const void* k_idx;
-  const void* q_idx;
+  const void* q_idx;            // [B * nq, d]
   int d;
   const int64_t* seq_start;
   float scale;
-  float* scores;
-  unsigned int* hist;
+  float* scores;                // query v's scores at score_base(v)
+  unsigned int* hist;           // [B * nq, kHistBins]
   const int* invalid;
   const int32_t* block_table;   // paged cache (PAGED kernels only)
   int bt_ld, bs_log2;
+  int nq;                       // new tokens per sequence
 };
+
+// Several new tokens per sequence: query j (0 .. nq-1) of sequence b is query
+// v = b * nq + j; it sits at position len_b - nq + j and sees the first
+// len_b - nq + 1 + j rows.  Its scores are stored from score_base(v) on: the
+// queries' score arrays follow one another in v order.
+__device__ __forceinline__ int64_t query_len(const int64_t* seq_start, int b, int j, int nq) {
+  return seq_start[b + 1] - seq_start[b] - (nq - 1 - j);
+}
+__device__ __forceinline__ int64_t score_base(const int64_t* seq_start, int b, int j, int nq) {
+  const int64_t len = seq_start[b + 1] - seq_start[b];
+  return static_cast<int64_t>(nq) * seq_start[b] - static_cast<int64_t>(b) * (nq * (nq - 1) / 2) +
+         static_cast<int64_t>(j) * (len - nq + 1) + j * (j - 1) / 2;
+}
 
 // Cache row of row s of sequence b in a paged cache.
 __device__ __forceinline__ int64_t paged_row(const ScanParams& p, int b, int64_t s) {
@@ -206,12 +221,16 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
 // PAGED: the cache is block-paged; the CTA's slice of its sequence's block
 // table (at most kScanRowsPerCta entries, block sizes being powers of two) is
 // staged in shared memory, and each row address is looked up there.
-template <int ESIZE, int LPR, bool PAGED>
+//
+// NQ > 1: the sequence's NQ new tokens are scored against each row at once,
+// so the index cache is read once for all of them; query j keeps the rows
+// before its position only.
+template <int ESIZE, int LPR, bool PAGED, int NQ>
 __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const ScanParams p) {
   constexpr int RPL = 32 / LPR;                 // rows per warp load
   constexpr int U = 8;                          // loads in flight per lane
   constexpr int VALS = 16 / ESIZE;              // index values per 16-byte slice
-  __shared__ unsigned int hist[kHistBins];
+  __shared__ unsigned int hist[NQ][kHistBins];
   __shared__ int32_t blk[PAGED ? kScanRowsPerCta : 1];
   if (*p.invalid) return;
   const int b = blockIdx.y;
@@ -222,18 +241,25 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   const int64_t c1 = min64(len, c0 + kScanRowsPerCta);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPR, rsub = lane / LPR;
-  float qv[VALS];
+  float qv[NQ][VALS];
 #pragma unroll
-  for (int i = 0; i < VALS; ++i) {
-    const int j = sub * VALS + i;
-    if (ESIZE == 1) {
-      const __nv_fp8_storage_t v = static_cast<const __nv_fp8_storage_t*>(p.q_idx)[b * p.d + j];
-      qv[i] = __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)));
-    } else {
-      qv[i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q_idx)[b * p.d + j]);
+  for (int t = 0; t < NQ; ++t) {
+    const int64_t qrow = static_cast<int64_t>(b) * NQ + t;
+#pragma unroll
+    for (int i = 0; i < VALS; ++i) {
+      const int j = sub * VALS + i;
+      if (ESIZE == 1) {
+        const __nv_fp8_storage_t v = static_cast<const __nv_fp8_storage_t*>(p.q_idx)[qrow * p.d + j];
+        qv[t][i] = __half2float(__half(__nv_cvt_fp8_to_halfraw(v, __NV_E4M3)));
+      } else {
+        qv[t][i] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q_idx)[qrow * p.d + j]);
+      }
     }
   }
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  int64_t sbase[NQ];
+#pragma unroll
+  for (int t = 0; t < NQ; ++t) sbase[t] = score_base(p.seq_start, b, t, NQ);
+  for (int i = threadIdx.x; i < NQ * kHistBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   const int64_t j0 = PAGED ? c0 >> p.bs_log2 : 0;
   const int64_t off_mask = (int64_t(1) << p.bs_log2) - 1;
   if (PAGED) {
@@ -274,7 +300,9 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-      float acc = 0.0f;
+      float acc[NQ];
+#pragma unroll
+      for (int t = 0; t < NQ; ++t) acc[t] = 0.0f;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         if (ESIZE == 1) {
@@ -283,30 +311,45 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
             const __nv_fp8x2_storage_t pair =
                 static_cast<__nv_fp8x2_storage_t>((words[k] >> (16 * h)) & 0xFFFFu);
             const float2 f = __half22float2(__half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3)));
-            acc = fmaf(qv[4 * k + 2 * h], f.x, acc);
-            acc = fmaf(qv[4 * k + 2 * h + 1], f.y, acc);
+#pragma unroll
+            for (int t = 0; t < NQ; ++t) {
+              acc[t] = fmaf(qv[t][4 * k + 2 * h], f.x, acc[t]);
+              acc[t] = fmaf(qv[t][4 * k + 2 * h + 1], f.y, acc[t]);
+            }
           }
         } else {
           const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&words[k]));
-          acc = fmaf(qv[2 * k], f.x, acc);
-          acc = fmaf(qv[2 * k + 1], f.y, acc);
+#pragma unroll
+          for (int t = 0; t < NQ; ++t) {
+            acc[t] = fmaf(qv[t][2 * k], f.x, acc[t]);
+            acc[t] = fmaf(qv[t][2 * k + 1], f.y, acc[t]);
+          }
         }
       }
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+      for (int t = 0; t < NQ; ++t)
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xFFFFFFFFu, acc[t], o);
       const int64_t r = r0 + u * RPL + rsub;
       if (sub == 0 && r < c1) {
-        float sc = __fmul_rn(acc, p.scale);
-        sc = sc > 0.0f ? sc : 0.0f;
-        p.scores[base + r] = sc;
-        const uint32_t bin = __float_as_uint(sc) >> 20;
-        if (bin) atomicAdd(&hist[bin], 1u);  // zero scores are recovered by the select
+#pragma unroll
+        for (int t = 0; t < NQ; ++t) {
+          if (r < len - (NQ - 1 - t)) {   // causal for query t
+            float sc = __fmul_rn(acc[t], p.scale);
+            sc = sc > 0.0f ? sc : 0.0f;
+            p.scores[sbase[t] + r] = sc;
+            const uint32_t bin = __float_as_uint(sc) >> 20;
+            if (bin) atomicAdd(&hist[t][bin], 1u);  // zero scores are recovered by the select
+          }
+        }
       }
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
-    if (hist[i]) atomicAdd(&p.hist[static_cast<int64_t>(b) * kHistBins + i], hist[i]);
+  for (int i = threadIdx.x; i < NQ * kHistBins; i += blockDim.x) {
+    const unsigned int h = (&hist[0][0])[i];
+    if (h) atomicAdd(&p.hist[static_cast<int64_t>(b) * NQ * kHistBins + i], h);
+  }
 }
 
 // ---- select ------------------------------------------------------------------
@@ -386,8 +429,9 @@ struct DSelParams {
   const int64_t* seq_start;
   int top_k;
   int32_t* indices;
-  unsigned long long* scratch;   // [total_rows] (rows of sequence b at seq_start[b])
+  unsigned long long* scratch;   // [scores] (query v's keys from score_base(v) on)
   const int* invalid;
+  int nq;
 };
 
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelParams p) {
@@ -400,14 +444,14 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   int* sh = reinterpret_cast<int*>(wsum + 2 * kSelWarps);          // [8]
   unsigned int* h256 = dbase;                                      // fallback path histogram
   if (*p.invalid) return;
-  const int b = blockIdx.x;
+  const int v = blockIdx.x;                   // query v = b * nq + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t base = p.seq_start[b];
-  const int n = static_cast<int>(p.seq_start[b + 1] - base);
+  const int64_t base = score_base(p.seq_start, v / p.nq, v % p.nq, p.nq);
+  const int n = static_cast<int>(query_len(p.seq_start, v / p.nq, v % p.nq, p.nq));
   const int m = min(p.top_k, n);
   const float* sc = p.scores + base;
-  const unsigned int* hist = p.hist + static_cast<int64_t>(b) * kHistBins;
-  int32_t* out = p.indices + static_cast<int64_t>(b) * p.top_k;
+  const unsigned int* hist = p.hist + static_cast<int64_t>(v) * kHistBins;
+  int32_t* out = p.indices + static_cast<int64_t>(v) * p.top_k;
 
   // Bin of the m-th best score.  The histogram is staged in shared memory
   // (bufB is free until the sort); thread i owns bins 2047 - 2i and 2046 - 2i,
@@ -572,53 +616,70 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
     out[i] = i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
 }
 
-template <bool PAGED>
-void launch_scan(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
+template <bool PAGED, int NQ>
+bool launch_scan_rows(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
   if (esize == 1 && lpr == 8)
-    decode_scan_rows_kernel<1, 8, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 8, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 1 && lpr == 4)
-    decode_scan_rows_kernel<1, 4, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 4, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 1 && lpr == 16)
-    decode_scan_rows_kernel<1, 16, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 16, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 2 && lpr == 8)
-    decode_scan_rows_kernel<2, 8, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<2, 8, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 2 && lpr == 16)
-    decode_scan_rows_kernel<2, 16, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
-  else if (esize == 1)
-    decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<2, 16, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
   else
-    decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    return false;
+  return true;
+}
+
+// Returns false when no kernel serves these rows (several new tokens with an
+// index row that is not 64, 128 or 256 bytes).
+template <bool PAGED>
+bool launch_scan(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
+  switch (sp.nq) {
+    case 1:
+      if (launch_scan_rows<PAGED, 1>(sp, grid, esize, lpr, stream)) return true;
+      if (esize == 1)
+        decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+      else
+        decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+      return true;
+    case 2: return launch_scan_rows<PAGED, 2>(sp, grid, esize, lpr, stream);
+    case 3: return launch_scan_rows<PAGED, 3>(sp, grid, esize, lpr, stream);
+    case 4: return launch_scan_rows<PAGED, 4>(sp, grid, esize, lpr, stream);
+    default: return false;
+  }
 }
 
 }  // namespace
 
 dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
-  if (cudaMemsetAsync(a.hist, 0, sizeof(unsigned int) * kHistBins * a.B, stream) != cudaSuccess)
+  if (cudaMemsetAsync(a.hist, 0, sizeof(unsigned int) * kHistBins * a.B * a.nq, stream) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (a.seq_lens)
-    validate_paged_kernel<<<a.B, 256, 0, stream>>>(a.seq_lens, a.B, a.max_len, a.block_table,
+    validate_paged_kernel<<<a.B, 256, 0, stream>>>(a.seq_lens, a.B, a.max_len, a.nq, a.block_table,
                                                    a.bt_ld, a.bs_log2, a.num_blocks,
                                                    a.seq_start_out, a.invalid);
   else
-    validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.invalid);
-  ScanParams sp{a.k_idx,   a.q_idx,   a.d,           a.seq_start, a.scale, a.scores,
-                a.hist,    a.invalid, a.block_table, a.bt_ld,     a.bs_log2};
+    validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.nq, a.invalid);
+  ScanParams sp{a.k_idx,   a.q_idx,   a.d,           a.seq_start, a.scale,    a.scores,
+                a.hist,    a.invalid, a.block_table, a.bt_ld,     a.bs_log2, a.nq};
   const dim3 grid(static_cast<unsigned int>((a.max_len + kScanRowsPerCta - 1) / kScanRowsPerCta),
                   static_cast<unsigned int>(a.B));
   const int lpr = a.d * a.esize / 16;  // 16-byte slices per index row
-  if (a.seq_lens)
-    launch_scan<true>(sp, grid, a.esize, lpr, stream);
-  else
-    launch_scan<false>(sp, grid, a.esize, lpr, stream);
+  const bool launched = a.seq_lens ? launch_scan<true>(sp, grid, a.esize, lpr, stream)
+                                   : launch_scan<false>(sp, grid, a.esize, lpr, stream);
+  if (!launched) return DSA_ERR_UNSUPPORTED;   // checked by the caller before any launch
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
 
-  DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid};
+  DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid, a.nq};
   const size_t smem = static_cast<size_t>(2 * kSmemKeys) * 8 +
                       (kSelWarps * 256 + 256 + 2 * kSelWarps + 8) * 4;
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  decode_select_kernel<<<a.B, kSelThreads, smem, stream>>>(dp);
+  decode_select_kernel<<<a.B * a.nq, kSelThreads, smem, stream>>>(dp);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 

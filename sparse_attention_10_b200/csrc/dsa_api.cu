@@ -106,30 +106,34 @@ PrefillPlan plan_prefill(int64_t L, int top_k, int64_t Lk) {
 // that is 4 splits, which timed 15% faster than 8 (two waves of shorter items).
 constexpr int kDecodeSplits = 8;
 
-static int decode_splits(int B) {
-  return std::clamp(2 * num_sms() / std::max(B, 1), 2, kDecodeSplits);
+static int decode_splits(int queries) {
+  return std::clamp(2 * num_sms() / std::max(queries, 1), 2, kDecodeSplits);
 }
 
 struct DecodePlan {
   size_t off_counters, off_scores, off_hist, off_keys, off_indices, off_part, off_seq, total;
 };
 
-// paged: one more array, the running sum of the lengths [B + 1] (int64)
-DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k, bool paged = false) {
+// paged: one more array, the running sum of the lengths [B + 1] (int64).
+// nq new tokens per sequence: B * nq queries, at most nq * total_rows scores.
+DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k, bool paged = false,
+                       int nq = 1) {
   DecodePlan p{};
+  const size_t nqry = static_cast<size_t>(B) * nq;
+  const size_t nscore = static_cast<size_t>(total_rows) * nq;
   size_t o = 0;
   p.off_counters = o;
   o = align_up(o + 64 * sizeof(int));
   p.off_scores = o;
-  o = align_up(o + total_rows * sizeof(float));
+  o = align_up(o + nscore * sizeof(float));
   p.off_hist = o;
-  o = align_up(o + static_cast<size_t>(B) * 2048 * sizeof(unsigned int));
+  o = align_up(o + nqry * 2048 * sizeof(unsigned int));
   p.off_keys = o;
-  o = align_up(o + total_rows * sizeof(unsigned long long));
+  o = align_up(o + nscore * sizeof(unsigned long long));
   p.off_indices = o;
-  o = align_up(o + static_cast<size_t>(B) * top_k * sizeof(int32_t));
+  o = align_up(o + nqry * top_k * sizeof(int32_t));
   p.off_part = o;
-  o = align_up(o + static_cast<size_t>(B) * kDecodeSplits * H * (D + 2) * sizeof(float));
+  o = align_up(o + nqry * kDecodeSplits * H * (D + 2) * sizeof(float));
   if (paged) {
     p.off_seq = o;
     o = align_up(o + static_cast<size_t>(B + 1) * sizeof(int64_t));
@@ -214,6 +218,7 @@ struct DecodeCall {
   int bt_ld, bs_log2;
   int64_t num_blocks;
   int B;
+  int nq;                        // new tokens per sequence (the last nq rows of each)
   int64_t total_rows;            // rows the workspace is planned for
   int64_t max_len;
   int idx_dtype, d_idx, D;
@@ -243,7 +248,9 @@ dsa_status run_decode(const DecodeCall& c) {
   if (c.D != 64 && c.D != 128) return DSA_ERR_UNSUPPORTED;
   dsa_status st = check_index_dims(c.idx_dtype, c.d_idx);
   if (st != DSA_OK) return st;
-  const DecodePlan plan = plan_decode(c.B, c.total_rows, c.H, c.D, c.top_k, paged);
+  if (c.nq < 1 || c.nq > 4 || static_cast<int64_t>(c.B) * c.nq > kMaxDecodeBatch) return DSA_ERR_INVALID_ARG;
+  if (!decode_nq_supported(c.nq, esize_of(c.idx_dtype), c.d_idx)) return DSA_ERR_UNSUPPORTED;
+  const DecodePlan plan = plan_decode(c.B, c.total_rows, c.H, c.D, c.top_k, paged, c.nq);
   if (c.workspace_bytes < plan.total) return DSA_ERR_WORKSPACE;
   cudaStream_t s = c.stream;
   uint8_t* ws = static_cast<uint8_t*>(c.workspace);
@@ -275,6 +282,7 @@ dsa_status run_decode(const DecodeCall& c) {
   dl.bs_log2 = c.bs_log2;
   dl.num_blocks = c.num_blocks;
   dl.seq_start_out = seq_ws;
+  dl.nq = c.nq;
   {
     StageScope scope(5, 3, s);  // validate + scan + select (timed together)
     if ((st = launch_decode_select(dl, s)) != DSA_OK) return st;
@@ -287,13 +295,14 @@ dsa_status run_decode(const DecodeCall& c) {
   at.kv_rows = paged ? c.num_blocks << c.bs_log2 : c.total_rows;
   at.idx = idx;
   at.ld_idx = c.top_k;
-  at.nq = c.B;
+  at.nq = static_cast<int64_t>(c.B) * c.nq;
+  at.qpt = c.nq;
   at.H = c.H;
   at.D = c.D;
   at.scale_log2 = default_scale(c.attn_scale, c.D) * 1.4426950408889634f;
   at.top_k = c.top_k;
   at.seq_start = seq_start;
-  at.nsplit = decode_splits(c.B);
+  at.nsplit = decode_splits(c.B * c.nq);
   at.O = static_cast<__nv_bfloat16*>(c.O);
   at.part = reinterpret_cast<float*>(ws + plan.off_part);
   at.invalid = dl.invalid;
@@ -500,9 +509,14 @@ dsa_status dsa_prefill_chunk(const void* q_idx, const void* k_idx, int idx_dtype
 
 size_t dsa_decode_workspace_size(int B, int64_t total_rows, int d_idx, int idx_dtype, int H,
                                  int D, int top_k) {
+  return dsa_decode_multi_workspace_size(B, 1, total_rows, d_idx, idx_dtype, H, D, top_k);
+}
+
+size_t dsa_decode_multi_workspace_size(int B, int T, int64_t total_rows, int d_idx, int idx_dtype,
+                                       int H, int D, int top_k) {
   (void)d_idx; (void)idx_dtype;
-  if (B < 1 || total_rows < 1 || H < 1 || top_k < 1) return 0;
-  return plan_decode(B, total_rows, H, D, top_k).total;
+  if (B < 1 || T < 1 || T > 4 || total_rows < 1 || H < 1 || top_k < 1) return 0;
+  return plan_decode(B, total_rows, H, D, top_k, false, T).total;
 }
 
 dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int64_t* seq_start,
@@ -510,6 +524,17 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
                       const void* q_idx, const void* Q, int H, int top_k, float idx_scale,
                       float attn_scale, void* O, int32_t* indices, void* workspace,
                       size_t workspace_bytes, void* stream) {
+  return dsa_decode_multi(k_idx, K, V, seq_start, B, 1, total_rows, max_len, idx_dtype, d_idx, D,
+                          q_idx, Q, H, top_k, idx_scale, attn_scale, O, indices, workspace,
+                          workspace_bytes, stream);
+}
+
+dsa_status dsa_decode_multi(const void* k_idx, const void* K, const void* V,
+                            const int64_t* seq_start, int B, int T, int64_t total_rows,
+                            int64_t max_len, int idx_dtype, int d_idx, int D, const void* q_idx,
+                            const void* Q, int H, int top_k, float idx_scale, float attn_scale,
+                            void* O, int32_t* indices, void* workspace, size_t workspace_bytes,
+                            void* stream) {
   if (!seq_start || (reinterpret_cast<uintptr_t>(seq_start) & 7) != 0 || total_rows < 1)
     return DSA_ERR_INVALID_ARG;
   DecodeCall c{};
@@ -518,6 +543,7 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
   c.V = V;
   c.seq_start = seq_start;
   c.B = B;
+  c.nq = T;
   c.total_rows = total_rows;
   c.max_len = max_len;
   c.idx_dtype = idx_dtype;
@@ -539,9 +565,15 @@ dsa_status dsa_decode(const void* k_idx, const void* K, const void* V, const int
 
 size_t dsa_decode_paged_workspace_size(int B, int64_t max_len, int d_idx, int idx_dtype, int H,
                                        int D, int top_k) {
+  return dsa_decode_paged_multi_workspace_size(B, 1, max_len, d_idx, idx_dtype, H, D, top_k);
+}
+
+size_t dsa_decode_paged_multi_workspace_size(int B, int T, int64_t max_len, int d_idx,
+                                             int idx_dtype, int H, int D, int top_k) {
   (void)d_idx; (void)idx_dtype;
-  if (B < 1 || max_len < 1 || max_len > kMaxDecodeLen || H < 1 || top_k < 1) return 0;
-  return plan_decode(B, static_cast<int64_t>(B) * max_len, H, D, top_k, true).total;
+  if (B < 1 || T < 1 || T > 4 || max_len < 1 || max_len > kMaxDecodeLen || H < 1 || top_k < 1)
+    return 0;
+  return plan_decode(B, static_cast<int64_t>(B) * max_len, H, D, top_k, true, T).total;
 }
 
 dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int64_t num_blocks,
@@ -550,6 +582,19 @@ dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int
                             int d_idx, int D, const void* q_idx, const void* Q, int H, int top_k,
                             float idx_scale, float attn_scale, void* O, int32_t* indices,
                             void* workspace, size_t workspace_bytes, void* stream) {
+  return dsa_decode_paged_multi(k_idx, K, V, num_blocks, block_size, block_table, max_blocks,
+                                seq_lens, B, 1, max_len, idx_dtype, d_idx, D, q_idx, Q, H, top_k,
+                                idx_scale, attn_scale, O, indices, workspace, workspace_bytes,
+                                stream);
+}
+
+dsa_status dsa_decode_paged_multi(const void* k_idx, const void* K, const void* V,
+                                  int64_t num_blocks, int block_size, const int32_t* block_table,
+                                  int max_blocks, const int32_t* seq_lens, int B, int T,
+                                  int64_t max_len, int idx_dtype, int d_idx, int D,
+                                  const void* q_idx, const void* Q, int H, int top_k,
+                                  float idx_scale, float attn_scale, void* O, int32_t* indices,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
   if (!block_table || !seq_lens || (reinterpret_cast<uintptr_t>(block_table) & 3) != 0 ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3) != 0)
     return DSA_ERR_INVALID_ARG;
@@ -570,6 +615,7 @@ dsa_status dsa_decode_paged(const void* k_idx, const void* K, const void* V, int
   c.bs_log2 = lg;
   c.num_blocks = num_blocks;
   c.B = B;
+  c.nq = T;
   c.total_rows = static_cast<int64_t>(B) * max_len;
   c.max_len = max_len;
   c.idx_dtype = idx_dtype;

@@ -101,6 +101,8 @@ struct AttnLaunch {
   const int32_t* block_table;
   int bt_ld, bs_log2;
   int64_t q0;                  // prefill: query q sits at key position q0 + q (chunked prefill)
+  int qpt;                     // decode: queries per sequence (query q belongs to sequence
+                               // q / qpt and sees its first len - (qpt - 1 - q % qpt) rows)
 };
 
 dsa_status launch_attention(const AttnLaunch& a, cudaStream_t stream);
@@ -135,9 +137,20 @@ struct DecodeLaunch {
   int bt_ld, bs_log2;
   int64_t num_blocks;
   int64_t* seq_start_out;
+  // nq new tokens per sequence (1 .. 4): query v = b * nq + j sits at position
+  // len_b - nq + j; q_idx is [B * nq, d], scores, histograms and indices are
+  // per query v (scores of query v from nq * seq_start[b] - b * nq(nq-1)/2 +
+  // j (len_b - nq + 1) + j(j-1)/2 on).  nq > 1 needs index rows of 64, 128 or
+  // 256 bytes (decode_nq_supported).
+  int nq;
 };
 
 dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream);
+inline bool decode_nq_supported(int nq, int esize, int d) {
+  const int lpr = d * esize / 16;
+  if (nq == 1) return true;
+  return nq >= 2 && nq <= 4 && (lpr == 4 || lpr == 8 || lpr == 16) && (esize == 1 || lpr != 4);
+}
 
 int num_sms();
 uint64_t wait_limit_ns();

@@ -178,6 +178,7 @@ WORKLOADS = {
 # tensor ids inside a workload's streams
 _T_QIDX, _T_KIDX, _T_Q, _T_K, _T_V, _T_BOOST, _T_LEN = 1, 2, 3, 4, 5, 6, 7
 _T_PAGE, _T_PAD_KIDX, _T_PAD_K, _T_PAD_V = 8, 9, 10, 11
+_T_MQIDX, _T_MQ = 12, 13
 
 
 def _encode_ints(v: np.ndarray, idx_dtype: str) -> np.ndarray:
@@ -265,6 +266,23 @@ def decode_inputs(w: Workload, seed: int = SEED, lengths: Optional[np.ndarray] =
         out["K"] = _prefix_normal(seed, w.cid, _T_K, total * w.D).reshape(total, w.D)
         out["V"] = _prefix_normal(seed, w.cid, _T_V, total * w.D).reshape(total, w.D)
     return out
+
+
+def multi_queries(w: Workload, B: int, T: int, seed: int = SEED) -> dict:
+    """Queries of T new tokens per sequence for a decode batch: q_idx [B, T, d_idx]
+    (integers in [-4, 4], encoded as the workload's index type) and Q [B, T, H, D]
+    BF16 N(0, 1).  Token t of sequence b uses the t-th of T draws of its streams."""
+    qi = uniform_ints(stream_key(seed, w.cid, _T_MQIDX, T), B * T * w.d_idx).reshape(B, T, w.d_idx)
+    return {"q_idx": _encode_ints(qi, w.idx_dtype),
+            "Q": _prefix_normal(seed, w.cid, _T_MQ * 16 + T, B * T * w.H * w.D).reshape(B, T, w.H, w.D)}
+
+
+def multi_queries_torch(w: Workload, B: int, T: int, seed: int = SEED, device="cuda") -> dict:
+    """multi_queries drawn on a device (same numbers)."""
+    qi = uniform_ints_torch(stream_key(seed, w.cid, _T_MQIDX, T), B * T * w.d_idx, device=device)
+    return {"q_idx": _encode_ints_torch(qi.view(B, T, w.d_idx), w.idx_dtype),
+            "Q": normal_bf16_torch(stream_key(seed, w.cid, _T_MQ * 16 + T), B * T * w.H * w.D,
+                                   device=device).view(B, T, w.H, w.D)}
 
 
 def paged_layout(lengths, block_size: int, seed: int = SEED, spare_blocks: int = 3):

@@ -133,3 +133,27 @@ def test_paged_decode_writes_stay_inside_buffers(dsa, zero_q):
     assert g_idx.intact() and g_o.intact() and g_ws.intact()
     assert torch.equal(idx, ref_idx)
     assert torch.equal(O.view(torch.int16), ref_o.view(torch.int16))
+
+
+def test_paged_multi_token_decode_writes_stay_inside_buffers(dsa):
+    import dataclasses
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([4, 100, 2049, 9000], dtype=np.int64)
+    T = 4
+    xp = synth.paged_decode_inputs(w, lens, 16)
+    mq = synth.multi_queries(w, len(lens), T)
+    t = {n: dev(xp[n]) for n in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens")}
+    B, mx = len(lens), int(lens.max())
+    need = dsa.dsa_decode_paged_multi_workspace_size(B, T, mx, w.d_idx, 0, w.H, w.D, w.top_k)
+    g_idx, g_o, g_ws = Guarded(B * T * w.top_k * 4), Guarded(B * T * w.H * w.D * 2), Guarded(need)
+    args = (t["k_idx_blocks"], t["K_blocks"].view(torch.bfloat16), t["V_blocks"].view(torch.bfloat16),
+            t["block_table"], t["seq_lens"], dev(mq["q_idx"]), dev(mq["Q"]).view(torch.bfloat16), w.top_k, mx)
+    O, idx = dsa.dsa_decode_paged_multi(*args, O=g_o.tensor(torch.bfloat16, (B, T, w.H, w.D)),
+                                        indices=g_idx.tensor(torch.int32, (B, T, w.top_k)),
+                                        workspace=g_ws.tensor())
+    assert dsa.dsa_sync_status() == 0
+    ref_o, ref_idx = dsa.dsa_decode_paged_multi(*args)
+    assert dsa.dsa_sync_status() == 0
+    assert g_idx.intact() and g_o.intact() and g_ws.intact()
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(O.view(torch.int16), ref_o.view(torch.int16))

@@ -426,3 +426,38 @@ def test_scale_overrides_are_applied(oracle_mod):
     di, do = oracle_mod.decode(xd, "fp8", k)
     ei, eo = oracle_mod.decode(xd2, "fp8", k, attn_scale=1.0 / np.sqrt(xd["Q"].shape[2]) / 2)
     assert np.array_equal(ei, di) and np.array_equal(eo, do)
+
+
+# ---------------------------------------------------------------- several new tokens per sequence
+
+def test_decode_multi_token_equals_prefill_rows_at_its_position():
+    """Token j of sequence b (T new tokens, the last T rows of the sequence) is the
+    prefill query at position len_b - T + j of that sequence: checked against the
+    prefill oracle on the sequence's own rows, and T = 1 is the single-token decode."""
+    import numpy as np
+    import oracle
+    import synth
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([4, 40, 300, 1000], dtype=np.int64)
+    T = 3
+    xd = synth.decode_inputs(w, lengths=lens)
+    mq = synth.multi_queries(w, len(lens), T)
+    x = dict(xd, q_idx=mq["q_idx"], Q=mq["Q"])
+    idx, O = oracle.decode_multi(x, w.idx_dtype, 128)
+    ss = xd["seq_start"]
+    for b, n in enumerate(lens):
+        rows = slice(ss[b], ss[b + 1])
+        for j in range(T):
+            pos = int(n) - T + j
+            qf = np.zeros((int(n), w.d_idx), dtype=xd["k_idx"].dtype)
+            qf[pos] = mq["q_idx"][b, j]
+            Qf = np.zeros((int(n), w.H, w.D), dtype=np.uint16)
+            Qf[pos] = mq["Q"][b, j]
+            p = {"q_idx": qf, "k_idx": xd["k_idx"][rows], "Q": Qf, "K": xd["K"][rows], "V": xd["V"][rows]}
+            ri, ro = oracle.prefill_rows(p, w.idx_dtype, 128, rows=np.array([pos], dtype=np.int64))
+            assert np.array_equal(idx[b, j], ri[0]), (b, j)
+            assert np.array_equal(O[b, j], ro[0]), (b, j)
+    x1 = dict(xd, q_idx=xd["q_idx"][:, None, :], Q=xd["Q"][:, None])
+    i1, o1 = oracle.decode_multi(x1, w.idx_dtype, 128)
+    i0, o0 = oracle.decode(xd, w.idx_dtype, 128)
+    assert np.array_equal(i1[:, 0], i0) and np.array_equal(o1[:, 0], o0)

@@ -539,6 +539,97 @@ def test_decode_wide_ties_many_candidates(dsa, mode, lens):
             assert idx[b, :m].tolist() == list(range(m))
 
 
+# ------------------------------------------------------------------ several new tokens per sequence
+
+def multi_case(lens, T, idx_dtype="fp8", d=128, D=128, seed=None):
+    import dataclasses
+    w = dataclasses.replace(synth.WORKLOADS["decode_64x128k"], d_idx=d, idx_dtype=idx_dtype, D=D)
+    lens = np.array(lens, dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    mq = synth.multi_queries(w, len(lens), T)
+    return w, dict(xd, q_idx=mq["q_idx"], Q=mq["Q"])
+
+
+@pytest.mark.parametrize("T,idx_dtype,d,D,top_k,lens", [
+    (2, "fp8", 128, 128, 2048, [2, 3, 100, 2049, 9000, 70000]),
+    (4, "fp8", 128, 128, 512, [4, 5, 2048, 4100, 30000]),
+    (3, "fp8", 64, 64, 300, [3, 777, 5000]),          # 64-byte index rows, head dim 64
+    (4, "bf16", 64, 128, 1024, [4, 1500, 20000]),     # BF16 index rows of 128 bytes
+])
+def test_decode_multi_matches_oracle(dsa, T, idx_dtype, d, D, top_k, lens):
+    w, x = multi_case(lens, T, idx_dtype, d, D)
+    t = {k: to_dev(x[k]) for k in ("k_idx", "K", "V", "q_idx", "Q", "seq_start")}
+    O, idx = dsa.dsa_decode_multi(t["k_idx"], t["K"].view(torch.bfloat16), t["V"].view(torch.bfloat16),
+                                  t["seq_start"], t["q_idx"], t["Q"].view(torch.bfloat16), top_k, max(lens))
+    assert dsa.dsa_sync_status() == 0
+    ri, ro = oracle.decode_multi(x, idx_dtype, top_k)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    got = O.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL
+
+
+@pytest.mark.parametrize("T,block_size", [(2, 64), (4, 16), (3, 1)])
+def test_decode_paged_multi_matches_oracle(dsa, T, block_size):
+    w, x = multi_case([3, 64, 2049, 20001], T)
+    xp = synth.paged_decode_inputs(w, x["lengths"], block_size)
+    t = {k: to_dev(xp[k]) for k in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens")}
+    O, idx = dsa.dsa_decode_paged_multi(t["k_idx_blocks"], t["K_blocks"].view(torch.bfloat16),
+                                        t["V_blocks"].view(torch.bfloat16), t["block_table"], t["seq_lens"],
+                                        to_dev(x["q_idx"]), bf16(x["Q"]), w.top_k, int(x["lengths"].max()))
+    assert dsa.dsa_sync_status() == 0
+    ri, ro = oracle.decode_multi(x, w.idx_dtype, w.top_k)
+    assert np.array_equal(idx.cpu().numpy(), ri)
+    got = O.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.abs(bits_to_f32(got) - bits_to_f32(ro)).max() <= ATOL
+
+
+def test_decode_multi_full_batch_equals_single_token_steps(dsa):
+    """The 64-sequence batch (65K-131K rows each) with T = 2: token 1 sees every row and
+    is the single-token decode of the same query; token 0 is the single-token decode of the
+    batch with each sequence's last row dropped."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    xd = synth.decode_inputs_torch(w, device="cuda")
+    mq = synth.multi_queries_torch(w, w.B, 2, device="cuda")
+    ss, lens = xd["seq_start"], xd["lengths"]
+    mx = int(lens.max())
+    O, idx = dsa.dsa_decode_multi(xd["k_idx"], xd["K"], xd["V"], ss, mq["q_idx"], mq["Q"], w.top_k, mx)
+    assert dsa.dsa_sync_status() == 0
+    O1, i1 = dsa.dsa_decode(xd["k_idx"], xd["K"], xd["V"], ss, mq["q_idx"][:, 1].contiguous(),
+                            mq["Q"][:, 1].contiguous(), w.top_k, mx)
+    assert torch.equal(idx[:, 1], i1)
+    assert (O[:, 1].float() - O1.float()).abs().max().item() <= ATOL
+    keep = torch.ones(xd["k_idx"].shape[0], dtype=torch.bool, device="cuda")
+    keep[ss[1:] - 1] = False                               # drop each sequence's last row
+    ss0 = ss - torch.arange(ss.shape[0], device="cuda", dtype=torch.int64)
+    O0, i0 = dsa.dsa_decode(xd["k_idx"][keep].contiguous(), xd["K"][keep].contiguous(), xd["V"][keep].contiguous(),
+                            ss0, mq["q_idx"][:, 0].contiguous(), mq["Q"][:, 0].contiguous(), w.top_k, mx)
+    assert dsa.dsa_sync_status() == 0
+    assert torch.equal(idx[:, 0], i0)
+    assert (O[:, 0].float() - O0.float()).abs().max().item() <= ATOL
+
+
+def test_decode_multi_checks(dsa):
+    import ctypes
+    lib = dsa.load()
+    w, x = multi_case([5, 9], 2, d=96)          # 96-byte FP8 index rows: no multi-token scan
+    t = {k: to_dev(x[k]) for k in ("k_idx", "K", "V", "q_idx", "Q", "seq_start")}
+    P = lambda a: ctypes.c_void_p(a.data_ptr())
+    args = lambda T: (P(t["k_idx"]), P(t["K"]), P(t["V"]), P(t["seq_start"]), 2, T, 14, 9, 0, 96, 128,
+                      P(t["q_idx"]), P(t["Q"]), 16, 64, float("nan"), float("nan"), P(t["Q"]), None)
+    ws = torch.empty(1 << 24, dtype=torch.uint8, device="cuda")
+    assert lib.dsa_decode_multi(*args(2), P(ws), ws.numel(), None) == 2   # DSA_ERR_UNSUPPORTED
+    assert lib.dsa_decode_multi(*args(5), P(ws), ws.numel(), None) == 1   # T outside [1, 4]
+    assert lib.dsa_decode_multi_workspace_size(2, 5, 14, 96, 0, 16, 128, 64) == 0
+    # lengths shorter than T are caught on the device: the call records DSA_ERR_INVALID_ARG
+    w, x = multi_case([1, 9], 1)
+    mq = synth.multi_queries(w, 2, 2)
+    t = {k: to_dev(x[k]) for k in ("k_idx", "K", "V", "seq_start")}
+    dsa.dsa_decode_multi(t["k_idx"], t["K"].view(torch.bfloat16), t["V"].view(torch.bfloat16), t["seq_start"],
+                         to_dev(mq["q_idx"]), bf16(mq["Q"]), 64, 9)
+    assert dsa.dsa_sync_status() == 1
+    assert dsa.dsa_sync_status() == 0
+
+
 # ------------------------------------------------------------------ paged decode
 
 def run_decode_paged(dsa, xp, top_k, max_len=None):
