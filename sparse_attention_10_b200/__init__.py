@@ -280,6 +280,16 @@ def dsa_decode_paged(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, bloc
     return O, indices
 
 
+def dsa_decode_multi_workspace_size(B: int, T: int, total_rows: int, d_idx: int, idx_dtype: int, H: int, D: int,
+                                    top_k: int) -> int:
+    return int(load().dsa_decode_multi_workspace_size(B, T, total_rows, d_idx, idx_dtype, H, D, top_k))
+
+
+def dsa_decode_paged_multi_workspace_size(B: int, T: int, max_len: int, d_idx: int, idx_dtype: int, H: int,
+                                          D: int, top_k: int) -> int:
+    return int(load().dsa_decode_paged_multi_workspace_size(B, T, max_len, d_idx, idx_dtype, H, D, top_k))
+
+
 def dsa_decode_multi(k_idx: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_start: torch.Tensor,
                      q_idx: torch.Tensor, Q: torch.Tensor, top_k: int, max_len: int,
                      idx_scale: Optional[float] = None, attn_scale: Optional[float] = None,

@@ -132,3 +132,8 @@ def test_force_fallback_hook_validates_and_resets(lib):
     assert lib.dsa_debug_force_fallback(-1) == 1     # negative period rejected
     dsa.dsa_debug_force_fallback(7)
     dsa.dsa_debug_force_fallback(0)                  # back to normal
+
+
+def test_binding_exports_what_it_lists():
+    import sparse_attention_10_b200 as m
+    assert [n for n in m.__all__ if not hasattr(m, n)] == []
