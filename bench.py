@@ -804,6 +804,42 @@ def main():
             "layout": f"k_idx/K/V pools of {xp['k_idx_blocks'].shape[0]} blocks x {bsz} rows, "
                       f"block table [{wd.B}, {xp['block_table'].shape[1]}] int32, seeded block order",
             "matches_contiguous": bool(torch.equal(idp, idd) and torch.equal(Op, Od))}
+
+        # several new tokens per sequence (speculative drafts / short chunks) over the same paged
+        # cache: T tokens of each sequence are scored in one pass over its index rows
+        decode["multi_token"] = {}
+        for T in (2, 4):
+            mq = synth.multi_queries_torch(wd, wd.B, T, seed=seed, device=dev)
+            wsm = torch.empty(dsa.dsa_decode_paged_multi_workspace_size(wd.B, T, int(lengths.max()), wd.d_idx, 0,
+                                                                        wd.H, wd.D, wd.top_k),
+                              dtype=torch.uint8, device=dev)
+            Om = torch.empty((wd.B, T, wd.H, wd.D), dtype=torch.bfloat16, device=dev)
+            idm = torch.empty((wd.B, T, wd.top_k), dtype=torch.int32, device=dev)
+
+            def mstep():
+                dsa.dsa_decode_paged_multi(xp["k_idx_blocks"], xp["K_blocks"], xp["V_blocks"], xp["block_table"],
+                                           xp["seq_lens"], mq["q_idx"], mq["Q"], wd.top_k, int(lengths.max()),
+                                           O=Om, indices=idm, workspace=wsm, stream=stream)
+
+            for _ in range(args.warmup):
+                mstep()
+            torch.cuda.synchronize()
+            barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(nd):
+                mstep()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            mms = max_over_ranks(e0.elapsed_time(e1))
+            if dsa.dsa_sync_status(stream) != 0:
+                raise RuntimeError("device-side error in multi-token decode")
+            decode["multi_token"][f"T{T}"] = {
+                "value": world * wd.B * T * nd / (mms / 1000.0), "unit": "tok/s", "ms_per_step": mms / nd,
+                "tokens_per_step": wd.B * T,
+                "how": f"dsa_decode_paged_multi, {T} new tokens per sequence, the paged cache above"}
+            del mq, wsm, Om, idm
         del xp, wsp
 
     # --- the other prefill workloads (4K, 32K and 64K), each timed on its own
