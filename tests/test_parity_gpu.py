@@ -570,7 +570,7 @@ def test_decode_multi_matches_oracle(dsa, T, idx_dtype, d, D, top_k, lens):
 
 @pytest.mark.parametrize("T,block_size", [(2, 64), (4, 16), (3, 1)])
 def test_decode_paged_multi_matches_oracle(dsa, T, block_size):
-    w, x = multi_case([3, 64, 2049, 20001], T)
+    w, x = multi_case([4, 64, 2049, 20001], T)       # every length >= T
     xp = synth.paged_decode_inputs(w, x["lengths"], block_size)
     t = {k: to_dev(xp[k]) for k in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens")}
     O, idx = dsa.dsa_decode_paged_multi(t["k_idx_blocks"], t["K_blocks"].view(torch.bfloat16),
