@@ -14,6 +14,7 @@
 // the m-th best score; every key at or above that bin is compacted into shared
 // memory (or, when too many, into a global scratch row) and the exact select
 // plus sort of the prefill path finishes the row.
+#include <cooperative_groups.h>
 #include <cuda_fp8.h>
 
 #include <algorithm>
@@ -434,7 +435,16 @@ struct DSelParams {
   int nq;
 };
 
-__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelParams p) {
+// A cluster of two CTAs per query: both find the boundary bin, each compacts
+// the candidates of one half of the query's scores (index order is kept: the
+// first CTA takes the lower half), and the first CTA gathers the second's list
+// from its shared memory (distributed shared memory) and finishes the select.
+constexpr int kSelCluster = 2;
+__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
+    decode_select_kernel(const DSelParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const unsigned int crank = cluster.block_rank();
   extern __shared__ unsigned long long ds_smem[];
   unsigned long long* bufA = ds_smem;                              // [kSmemKeys]
   unsigned long long* bufB = bufA + kSmemKeys;                     // [kSmemKeys]
@@ -444,7 +454,7 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   int* sh = reinterpret_cast<int*>(wsum + 2 * kSelWarps);          // [8]
   unsigned int* h256 = dbase;                                      // fallback path histogram
   if (*p.invalid) return;
-  const int v = blockIdx.x;                   // query v = b * nq + j
+  const int v = blockIdx.x / kSelCluster;     // query v = b * nq + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t base = score_base(p.seq_start, v / p.nq, v % p.nq, p.nq);
   const int n = static_cast<int>(query_len(p.seq_start, v / p.nq, v % p.nq, p.nq));
@@ -514,12 +524,15 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
     uint32_t o_or = 0u, o_and = 0xFFFFFFFFu;
     constexpr int kPer = 8;
     constexpr int kRound = kSelThreads * kPer;
-    const int rounds = (n + kRound - 1) / kRound;
+    const int half = ((n + 1) / 2 + kPer - 1) / kPer * kPer;
+    const int lo = crank ? min(n, half) : 0;      // this CTA's scores: [lo, hi)
+    const int hi = crank ? n : min(n, half);
+    const int rounds = (hi - lo + kRound - 1) / kRound;
     float vn[kPer];
     auto load = [&](int r) {
-      const int s = r * kRound + threadIdx.x * kPer;
+      const int s = lo + r * kRound + threadIdx.x * kPer;
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) vn[k] = s + k < n ? sc[s + k] : 0.0f;
+      for (int k = 0; k < kPer; ++k) vn[k] = s + k < hi ? sc[s + k] : 0.0f;
     };
     load(0);
     uint32_t done = 0;
@@ -528,11 +541,11 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
 #pragma unroll
       for (int k = 0; k < kPer; ++k) v[k] = vn[k];
       if (r + 1 < rounds) load(r + 1);
-      const int s = r * kRound + threadIdx.x * kPer;
+      const int s = lo + r * kRound + threadIdx.x * kPer;
       uint32_t flags = 0;
 #pragma unroll
       for (int k = 0; k < kPer; ++k)
-        if (s + k < n && (__float_as_uint(v[k]) >> 20) >= bin) flags |= 1u << k;
+        if (s + k < hi && (__float_as_uint(v[k]) >> 20) >= bin) flags |= 1u << k;
       const uint32_t c = __popc(flags);
       uint32_t incl = c;
 #pragma unroll
@@ -572,7 +585,22 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
       atomicOr(reinterpret_cast<unsigned int*>(&sh[3]), o_or);
       atomicAnd(reinterpret_cast<unsigned int*>(&sh[4]), o_and);
     }
-    __syncthreads();
+    cluster.sync();   // both halves compacted (also a barrier of each CTA)
+    if (crank == 0) {
+      const unsigned long long* rkeys = cluster.map_shared_rank(bufA, 1);
+      const int* rsh = cluster.map_shared_rank(sh, 1);
+      const int c0 = sh[2], c1 = rsh[2];
+      for (int i = threadIdx.x; i < c1; i += blockDim.x)
+        if (c0 + i < kSmemKeys) bufA[c0 + i] = rkeys[i];
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        sh[2] = c0 + c1;
+        sh[3] |= rsh[3];
+        sh[4] &= rsh[4];
+      }
+    }
+    cluster.sync();   // the second CTA's shared memory is no longer read
+    if (crank != 0) return;
     const int nc = min(sh[2], kSmemKeys);
     const uint32_t vary = static_cast<uint32_t>(sh[3]) ^ static_cast<uint32_t>(sh[4]);
     const unsigned long long* cur =
@@ -584,7 +612,9 @@ __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DSelPa
   }
 
   // Many candidates (wide ties): compact into the global scratch row, select
-  // the m-th key by radix passes there, then sort the m winners.
+  // the m-th key by radix passes there, then sort the m winners (first CTA of
+  // the cluster only).
+  if (crank != 0) return;
   unsigned long long* cand = p.scratch + base;
   if (threadIdx.x == 0) sh[2] = 0;
   __syncthreads();
@@ -679,7 +709,7 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
   if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return DSA_ERR_CUDA;
-  decode_select_kernel<<<a.B * a.nq, kSelThreads, smem, stream>>>(dp);
+  decode_select_kernel<<<a.B * a.nq * kSelCluster, kSelThreads, smem, stream>>>(dp);
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
