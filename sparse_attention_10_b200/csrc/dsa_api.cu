@@ -58,7 +58,7 @@ struct PrefillPlan {
   int samp_ld;
   int fb_ctas;
   size_t off_counters, off_tau, off_cand_n, off_cand, off_samp, off_fb_rows, off_fb_scratch,
-      off_fb_hist, off_fb_slow, total;
+      off_fb_hist, off_fb_slow, off_big_rows, total;
 };
 
 // L query rows against Lk key rows (Lk = L for a whole sequence).
@@ -95,6 +95,8 @@ PrefillPlan plan_prefill(int64_t L, int top_k, int64_t Lk) {
   o = align_up(o + static_cast<size_t>(p.fb_ctas) * 4096 * sizeof(unsigned int));
   p.off_fb_slow = o;
   o = align_up(o + static_cast<size_t>(p.fb_ctas) * sizeof(int));
+  p.off_big_rows = o;
+  o = align_up(o + L * sizeof(int));
   p.total = o;
   return p;
 }
@@ -480,10 +482,11 @@ dsa_status dsa_prefill_chunk(const void* q_idx, const void* k_idx, int idx_dtype
   sl.fb_scratch = fb_scratch;
   sl.fb_hist = reinterpret_cast<unsigned int*>(ws + plan.off_fb_hist);
   sl.fb_slow = reinterpret_cast<int*>(ws + plan.off_fb_slow);
+  sl.big_rows = reinterpret_cast<int*>(ws + plan.off_big_rows);
   sl.fb_ctas = plan.fb_ctas;
   sl.force_fb_period = g_force_fb_period.load();
   {
-    StageScope scope(3, 4, s);
+    StageScope scope(3, 5, s);
     if ((st = launch_select(sl, s)) != DSA_OK) return st;
   }
 

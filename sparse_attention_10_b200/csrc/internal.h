@@ -62,7 +62,8 @@ struct SelectLaunch {
   int* fb_rows;          // [L] rows that need the exact fallback
   int force_fb_period;   // > 0: rows t % period == 0 go to the fallback (test hook)
   int* counters;         // [0] fallback rows, [1] overflow rows, [2] candidates,
-                         // [3] fallback rows left to the one-CTA path
+                         // [3] fallback rows left to the one-CTA path, [4] big rows
+  int* big_rows;         // [L] rows whose candidates need the large select shape
   // fallback inputs
   const void* q_idx;
   const void* k_idx;

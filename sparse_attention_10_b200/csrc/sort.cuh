@@ -118,7 +118,8 @@ __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint3
                                  uint16_t* pout, int n, uint32_t kmin, int shift, int width,
                                  uint16_t* cnt16, uint32_t* base) {
   constexpr int kBins = 512;
-  static_assert(WARPS * 32 >= kBins, "one thread per digit");
+  constexpr int DPT = (kBins + WARPS * 32 - 1) / (WARPS * 32);   // digits per thread
+  static_assert(DPT * WARPS * 32 == kBins, "digits spread evenly over the threads");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = (n + WARPS * 32 - 1) / (WARPS * 32) * 32;  // items per warp
   const int slots = chunk / 32;
@@ -143,16 +144,21 @@ __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint3
     }
   }
   __syncthreads();
-  // per digit: exclusive prefix over the warps (in place), digit total
-  const int d = threadIdx.x;
-  uint32_t total = 0;
-  if (d < kBins) {
+  // per digit (thread t owns digits DPT t .. DPT t + DPT - 1): exclusive prefix
+  // over the warps (in place), digit totals
+  uint32_t tot[DPT], total = 0;
+#pragma unroll
+  for (int q = 0; q < DPT; ++q) {
+    const int d = DPT * threadIdx.x + q;
+    uint32_t run = 0;
 #pragma unroll 4
     for (int w = 0; w < WARPS; ++w) {
       const uint32_t c = cnt16[w * kBins + d];
-      cnt16[w * kBins + d] = static_cast<uint16_t>(total);
-      total += c;
+      cnt16[w * kBins + d] = static_cast<uint16_t>(run);
+      run += c;
     }
+    tot[q] = run;
+    total += run;
   }
   // exclusive scan of the digit totals over the block (digits in thread order)
   uint32_t incl = total;
@@ -163,10 +169,15 @@ __device__ void radix_pass32_var(const uint32_t* kin, const uint16_t* pin, uint3
   }
   if (lane == 31) base[kBins + warp] = incl;  // warp sums after the digit bases
   __syncthreads();
-  if (d < kBins) {
+  {
     uint32_t off = 0;
     for (int w = 0; w < warp; ++w) off += base[kBins + w];
-    base[d] = off + incl - total;
+    off += incl - total;
+#pragma unroll
+    for (int q = 0; q < DPT; ++q) {
+      base[DPT * threadIdx.x + q] = off;
+      off += tot[q];
+    }
   }
   __syncthreads();
 #pragma unroll
