@@ -435,12 +435,14 @@ struct DSelParams {
   int nq;
 };
 
-// A cluster of two CTAs per query: both find the boundary bin, each compacts
-// the candidates of one half of the query's scores (index order is kept: the
-// first CTA takes the lower half), and the first CTA gathers the second's list
-// from its shared memory (distributed shared memory) and finishes the select.
-constexpr int kSelCluster = 2;
-__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
+// CL = 2: a cluster of two CTAs per query: both find the boundary bin, each
+// compacts the candidates of one half of the query's scores (index order is
+// kept: the first CTA takes the lower half), and the first CTA gathers the
+// second's list from its shared memory (distributed shared memory) and
+// finishes the select.  CL = 1: one CTA per query (queries enough to fill
+// the GPU on their own, e.g. several new tokens per sequence).
+template <int CL>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kSelThreads)
     decode_select_kernel(const DSelParams p) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
@@ -454,7 +456,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
   int* sh = reinterpret_cast<int*>(wsum + 2 * kSelWarps);          // [8]
   unsigned int* h256 = dbase;                                      // fallback path histogram
   if (*p.invalid) return;
-  const int v = blockIdx.x / kSelCluster;     // query v = b * nq + j
+  const int v = blockIdx.x / CL;              // query v = b * nq + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t base = score_base(p.seq_start, v / p.nq, v % p.nq, p.nq);
   const int n = static_cast<int>(query_len(p.seq_start, v / p.nq, v % p.nq, p.nq));
@@ -526,7 +528,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
     constexpr int kRound = kSelThreads * kPer;
     const int half = ((n + 1) / 2 + kPer - 1) / kPer * kPer;
     const int lo = crank ? min(n, half) : 0;      // this CTA's scores: [lo, hi)
-    const int hi = crank ? n : min(n, half);
+    const int hi = (crank || CL == 1) ? n : min(n, half);
     const int rounds = (hi - lo + kRound - 1) / kRound;
     float vn[kPer];
     auto load = [&](int r) {
@@ -585,22 +587,26 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
       atomicOr(reinterpret_cast<unsigned int*>(&sh[3]), o_or);
       atomicAnd(reinterpret_cast<unsigned int*>(&sh[4]), o_and);
     }
-    cluster.sync();   // both halves compacted (also a barrier of each CTA)
-    if (crank == 0) {
-      const unsigned long long* rkeys = cluster.map_shared_rank(bufA, 1);
-      const int* rsh = cluster.map_shared_rank(sh, 1);
-      const int c0 = sh[2], c1 = rsh[2];
-      for (int i = threadIdx.x; i < c1; i += blockDim.x)
-        if (c0 + i < kSmemKeys) bufA[c0 + i] = rkeys[i];
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        sh[2] = c0 + c1;
-        sh[3] |= rsh[3];
-        sh[4] &= rsh[4];
+    if constexpr (CL == 2) {
+      cluster.sync();   // both halves compacted (also a barrier of each CTA)
+      if (crank == 0) {
+        const unsigned long long* rkeys = cluster.map_shared_rank(bufA, 1);
+        const int* rsh = cluster.map_shared_rank(sh, 1);
+        const int c0 = sh[2], c1 = rsh[2];
+        for (int i = threadIdx.x; i < c1; i += blockDim.x)
+          if (c0 + i < kSmemKeys) bufA[c0 + i] = rkeys[i];
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          sh[2] = c0 + c1;
+          sh[3] |= rsh[3];
+          sh[4] &= rsh[4];
+        }
       }
+      cluster.sync();   // the second CTA's shared memory is no longer read
+      if (crank != 0) return;
+    } else {
+      __syncthreads();
     }
-    cluster.sync();   // the second CTA's shared memory is no longer read
-    if (crank != 0) return;
     const int nc = min(sh[2], kSmemKeys);
     const uint32_t vary = static_cast<uint32_t>(sh[3]) ^ static_cast<uint32_t>(sh[4]);
     const unsigned long long* cur =
@@ -706,10 +712,19 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
   DSelParams dp{a.scores, a.hist, a.seq_start, a.top_k, a.indices, a.keys, a.invalid, a.nq};
   const size_t smem = static_cast<size_t>(2 * kSmemKeys) * 8 +
                       (kSelWarps * 256 + 256 + 2 * kSelWarps + 8) * 4;
-  if (cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  decode_select_kernel<<<a.B * a.nq * kSelCluster, kSelThreads, smem, stream>>>(dp);
+  // two CTAs per query while the queries fill at most half the SMs (one CTA per SM)
+  const int64_t queries = static_cast<int64_t>(a.B) * a.nq;
+  if (2 * queries <= num_sms()) {
+    if (cudaFuncSetAttribute(decode_select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    decode_select_kernel<2><<<static_cast<unsigned int>(2 * queries), kSelThreads, smem, stream>>>(dp);
+  } else {
+    if (cudaFuncSetAttribute(decode_select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    decode_select_kernel<1><<<static_cast<unsigned int>(queries), kSelThreads, smem, stream>>>(dp);
+  }
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
