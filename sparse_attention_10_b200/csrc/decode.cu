@@ -152,6 +152,7 @@ struct ScanParams {
   const int32_t* block_table;   // paged cache (PAGED kernels only)
   int bt_ld, bs_log2;
   int nq;                       // new tokens per sequence
+  int q_first;                  // multi-query scans: first of this launch's queries (0 .. nq-1)
 };
 
 // Several new tokens per sequence: query j (0 .. nq-1) of sequence b is query
@@ -223,10 +224,14 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
 // table (at most kScanRowsPerCta entries, block sizes being powers of two) is
 // staged in shared memory, and each row address is looked up there.
 //
-// NQ > 1: the sequence's NQ new tokens are scored against each row at once,
-// so the index cache is read once for all of them; query j keeps the rows
-// before its position only.
-template <int ESIZE, int LPR, bool PAGED, int NQ>
+// NQ > 1: NQ of the sequence's nq new tokens (q_first .. q_first + NQ - 1)
+// are scored against each row at once, so one pass over the index cache serves
+// them all; query j keeps the rows up to its position only.  Four queries per
+// thread need 148 registers (one CTA per SM) and ran slower than two passes of
+// two.  PASS: the launch is one of several (q_first and nq read at run time);
+// otherwise NQ is the whole count, which keeps the single-query kernel at 80
+// registers (three CTAs per SM).
+template <int ESIZE, int LPR, bool PAGED, int NQ, bool PASS>
 __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const ScanParams p) {
   constexpr int RPL = 32 / LPR;                 // rows per warp load
   constexpr int U = 8;                          // loads in flight per lane
@@ -242,10 +247,12 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   const int64_t c1 = min64(len, c0 + kScanRowsPerCta);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane % LPR, rsub = lane / LPR;
+  const int nq = PASS ? p.nq : NQ;
+  const int q_first = PASS ? p.q_first : 0;
   float qv[NQ][VALS];
 #pragma unroll
   for (int t = 0; t < NQ; ++t) {
-    const int64_t qrow = static_cast<int64_t>(b) * NQ + t;
+    const int64_t qrow = static_cast<int64_t>(b) * nq + q_first + t;
 #pragma unroll
     for (int i = 0; i < VALS; ++i) {
       const int j = sub * VALS + i;
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   }
   int64_t sbase[NQ];
 #pragma unroll
-  for (int t = 0; t < NQ; ++t) sbase[t] = score_base(p.seq_start, b, t, NQ);
+  for (int t = 0; t < NQ; ++t) sbase[t] = score_base(p.seq_start, b, q_first + t, nq);
   for (int i = threadIdx.x; i < NQ * kHistBins; i += blockDim.x) (&hist[0][0])[i] = 0;
   const int64_t j0 = PAGED ? c0 >> p.bs_log2 : 0;
   const int64_t off_mask = (int64_t(1) << p.bs_log2) - 1;
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
       if (sub == 0 && r < c1) {
 #pragma unroll
         for (int t = 0; t < NQ; ++t) {
-          if (r < len - (NQ - 1 - t)) {   // causal for query t
+          if (r < len - (nq - 1 - (q_first + t))) {   // causal for query q_first + t
             float sc = __fmul_rn(acc[t], p.scale);
             sc = sc > 0.0f ? sc : 0.0f;
             p.scores[sbase[t] + r] = sc;
@@ -349,7 +356,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   __syncthreads();
   for (int i = threadIdx.x; i < NQ * kHistBins; i += blockDim.x) {
     const unsigned int h = (&hist[0][0])[i];
-    if (h) atomicAdd(&p.hist[static_cast<int64_t>(b) * NQ * kHistBins + i], h);
+    if (h) atomicAdd(&p.hist[(static_cast<int64_t>(b) * nq + q_first) * kHistBins + i], h);
   }
 }
 
@@ -652,40 +659,45 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kSelThreads)
     out[i] = i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
 }
 
-template <bool PAGED, int NQ>
+template <bool PAGED, int NQ, bool PASS>
 bool launch_scan_rows(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
   if (esize == 1 && lpr == 8)
-    decode_scan_rows_kernel<1, 8, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 8, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 1 && lpr == 4)
-    decode_scan_rows_kernel<1, 4, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 4, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 1 && lpr == 16)
-    decode_scan_rows_kernel<1, 16, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<1, 16, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 2 && lpr == 8)
-    decode_scan_rows_kernel<2, 8, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<2, 8, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
   else if (esize == 2 && lpr == 16)
-    decode_scan_rows_kernel<2, 16, PAGED, NQ><<<grid, kScanThreads, 0, stream>>>(sp);
+    decode_scan_rows_kernel<2, 16, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
   else
     return false;
   return true;
 }
 
 // Returns false when no kernel serves these rows (several new tokens with an
-// index row that is not 64, 128 or 256 bytes).
+// index row that is not 64, 128 or 256 bytes).  Several tokens are scanned in
+// passes of two (and one for an odd count).
 template <bool PAGED>
-bool launch_scan(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
-  switch (sp.nq) {
-    case 1:
-      if (launch_scan_rows<PAGED, 1>(sp, grid, esize, lpr, stream)) return true;
-      if (esize == 1)
-        decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
-      else
-        decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
-      return true;
-    case 2: return launch_scan_rows<PAGED, 2>(sp, grid, esize, lpr, stream);
-    case 3: return launch_scan_rows<PAGED, 3>(sp, grid, esize, lpr, stream);
-    case 4: return launch_scan_rows<PAGED, 4>(sp, grid, esize, lpr, stream);
-    default: return false;
+bool launch_scan(ScanParams sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
+  sp.q_first = 0;
+  if (sp.nq == 2) return launch_scan_rows<PAGED, 2, false>(sp, grid, esize, lpr, stream);
+  if (sp.nq == 1) {
+    if (launch_scan_rows<PAGED, 1, false>(sp, grid, esize, lpr, stream)) return true;
+    if (esize == 1)
+      decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    else
+      decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+    return true;
   }
+  for (int q = 0; q < sp.nq; q += 2) {
+    sp.q_first = q;
+    const bool ok = q + 1 < sp.nq ? launch_scan_rows<PAGED, 2, true>(sp, grid, esize, lpr, stream)
+                                  : launch_scan_rows<PAGED, 1, true>(sp, grid, esize, lpr, stream);
+    if (!ok) return false;
+  }
+  return true;
 }
 
 }  // namespace
@@ -700,7 +712,7 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
   else
     validate_kernel<<<1, 256, 0, stream>>>(a.seq_start, a.B, a.total_rows, a.max_len, a.nq, a.invalid);
   ScanParams sp{a.k_idx,   a.q_idx,   a.d,           a.seq_start, a.scale,    a.scores,
-                a.hist,    a.invalid, a.block_table, a.bt_ld,     a.bs_log2, a.nq};
+                a.hist,    a.invalid, a.block_table, a.bt_ld,     a.bs_log2, a.nq, 0};
   const dim3 grid(static_cast<unsigned int>((a.max_len + kScanRowsPerCta - 1) / kScanRowsPerCta),
                   static_cast<unsigned int>(a.B));
   const int lpr = a.d * a.esize / 16;  // 16-byte slices per index row
