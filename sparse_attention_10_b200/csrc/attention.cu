@@ -126,6 +126,8 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
   const int g = lane >> 2, tig = lane & 3;
   const int64_t n_items = p.nq * p.nsplit;
 
+  griddep_wait();   // the select's indices
+  griddep_launch_dependents();
   if (p.invalid && *p.invalid) return;
   for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int64_t q = item / p.nsplit;
@@ -363,10 +365,29 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
   }
 }
 
+// Launch on `stream`; programmatic (may overlap the previous kernel's tail,
+// the kernel waiting on griddep_wait) when `pdl`.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_programmatic(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                      cudaStream_t stream, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Merge split partials: O = sum_s 2^(M_s - M) O_s / sum_s 2^(M_s - M) L_s.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(const float* part, int nsplit, int H,
                                                     __nv_bfloat16* O, const int* invalid) {
+  griddep_wait();   // the attention's partials
   if (invalid && *invalid) return;
   const int64_t qh = blockIdx.x;
   const int64_t q = qh / H, h = qh % H;
@@ -388,9 +409,10 @@ __global__ void __launch_bounds__(D) combine_kernel(const float* part, int nspli
 template <int D>
 dsa_status launch_combine(const AttnLaunch& a, cudaStream_t stream) {
   if (a.nsplit == 1) return DSA_OK;
-  combine_kernel<D><<<static_cast<unsigned int>(a.nq * a.H), D, 0, stream>>>(a.part, a.nsplit, a.H,
-                                                                             a.O, a.invalid);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  const cudaError_t e = launch_maybe_programmatic(combine_kernel<D>, dim3(static_cast<unsigned int>(a.nq * a.H)),
+                                                  dim3(D), 0, stream, a.seq_start != nullptr, a.part,
+                                                  a.nsplit, a.H, a.O, a.invalid);
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 template <int D>
@@ -409,8 +431,10 @@ dsa_status launch_d(const AttnLaunch& a, cudaStream_t stream) {
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_kernel<D>, kAttnThreads, smem);
   const int64_t items = a.nq * a.nsplit;
   const int grid = static_cast<int>(std::min<int64_t>(items, std::max(1, per_sm) * num_sms()));
-  attn_kernel<D><<<grid, kAttnThreads, smem, stream>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  // decode (seq_start set) follows the select kernel: launched programmatically
+  const cudaError_t e2 = launch_maybe_programmatic(attn_kernel<D>, dim3(grid), dim3(kAttnThreads), smem, stream,
+                                                   a.seq_start != nullptr, p);
+  if (e2 != cudaSuccess || cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   return launch_combine<D>(a, stream);
 }
 

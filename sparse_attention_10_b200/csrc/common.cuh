@@ -37,6 +37,18 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Bound on a single device-side wait (nanoseconds).
 __device__ __forceinline__ uint64_t wait_limit_ns_device() { return 2000000000ull; }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel of the stream finishes; it waits here, before reading
+// anything, until that kernel has completed and its writes are visible.
+// Without such a launch both are no-ops.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel of the stream (if launched programmatically) be
+// scheduled once every CTA of this grid has started.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

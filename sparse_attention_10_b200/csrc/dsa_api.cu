@@ -126,10 +126,10 @@ DecodePlan plan_decode(int B, int64_t total_rows, int H, int D, int top_k, bool 
   size_t o = 0;
   p.off_counters = o;
   o = align_up(o + 64 * sizeof(int));
+  p.off_hist = o;   // right after the counters: one memset clears both
+  o = align_up(o + nqry * 2048 * sizeof(unsigned int));
   p.off_scores = o;
   o = align_up(o + nscore * sizeof(float));
-  p.off_hist = o;
-  o = align_up(o + nqry * 2048 * sizeof(unsigned int));
   p.off_keys = o;
   o = align_up(o + nscore * sizeof(unsigned long long));
   p.off_indices = o;
@@ -257,7 +257,8 @@ dsa_status run_decode(const DecodeCall& c) {
   cudaStream_t s = c.stream;
   uint8_t* ws = static_cast<uint8_t*>(c.workspace);
   int32_t* idx = c.indices ? c.indices : reinterpret_cast<int32_t*>(ws + plan.off_indices);
-  if (cudaMemsetAsync(ws + plan.off_counters, 0, 64 * sizeof(int), s) != cudaSuccess)
+  const size_t cleared = plan.off_hist + static_cast<size_t>(c.B) * c.nq * 2048 * sizeof(unsigned int);
+  if (cudaMemsetAsync(ws + plan.off_counters, 0, cleared - plan.off_counters, s) != cudaSuccess)
     return DSA_ERR_CUDA;
   int64_t* seq_ws = paged ? reinterpret_cast<int64_t*>(ws + plan.off_seq) : nullptr;
   const int64_t* seq_start = paged ? seq_ws : c.seq_start;
