@@ -365,24 +365,6 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(const AttnParams p) 
   }
 }
 
-// Launch on `stream`; programmatic (may overlap the previous kernel's tail,
-// the kernel waiting on griddep_wait) when `pdl`.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_maybe_programmatic(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                      cudaStream_t stream, bool pdl, Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
 // Merge split partials: O = sum_s 2^(M_s - M) O_s / sum_s 2^(M_s - M) L_s.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(const float* part, int nsplit, int H,

@@ -16,11 +16,11 @@
 // when too many, into a global scratch row) and the exact select plus sort of
 // the prefill path finishes the row.
 //
-// scan -> select -> attention -> combine are launched programmatically: each
-// kernel lets the next one's CTAs be placed once all of its own have started,
-// and the next one waits (griddepcontrol.wait) before reading anything.  With
-// the histograms cleared by the counters' memset this took the 64-sequence
-// decode step from 0.2246 to 0.2191 ms.
+// validate -> scan -> select -> attention -> combine are launched
+// programmatically: each kernel lets the next one's CTAs be placed once all of
+// its own have started, and the next one waits (griddepcontrol.wait) before
+// reading anything.  With the histograms cleared by the counters' memset this
+// took the 64-sequence decode step from 0.2246 to 0.2170 ms.
 #include <cooperative_groups.h>
 #include <cuda_fp8.h>
 
@@ -97,6 +97,7 @@ __device__ __forceinline__ float dot_row(const float* q, const void* base, int64
 // (nq new tokens per sequence sit at its last nq rows).
 __global__ void validate_kernel(const int64_t* seq_start, int B, int64_t total_rows,
                                 int64_t max_len, int nq, int* invalid) {
+  griddep_launch_dependents();
   bool bad = false;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int64_t len = seq_start[b + 1] - seq_start[b];
@@ -117,6 +118,7 @@ __global__ void validate_paged_kernel(const int32_t* seq_lens, int B, int64_t ma
                                       const int32_t* table, int bt_ld, int bs_log2,
                                       int64_t num_blocks, int64_t* seq_start_out, int* invalid) {
   __shared__ long long wsum[32];
+  griddep_launch_dependents();
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   long long before = 0;
@@ -186,6 +188,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_kernel(const ScanPar
   __shared__ float qf[DSA_MAX_INDEX_DIM];
   __shared__ unsigned int hist[kHistBins];
   griddep_launch_dependents();
+  griddep_wait();   // the validation
   if (*p.invalid) return;
   const int b = blockIdx.y;
   const int64_t base = p.seq_start[b];
@@ -247,6 +250,7 @@ __global__ void __launch_bounds__(kScanThreads) decode_scan_rows_kernel(const Sc
   __shared__ unsigned int hist[NQ][kHistBins];
   __shared__ int32_t blk[PAGED ? kScanRowsPerCta : 1];
   griddep_launch_dependents();
+  griddep_wait();   // the validation (and, for a later pass, nothing: launched plainly)
   if (*p.invalid) return;
   const int b = blockIdx.y;
   const int64_t base = p.seq_start[b];
@@ -670,18 +674,20 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kSelThreads)
     out[i] = i < m ? static_cast<int32_t>(0xFFFFFFFFu - static_cast<uint32_t>(sel[i])) : -1;
 }
 
+// pdl: launched programmatically after the validation kernel (first pass only)
 template <bool PAGED, int NQ, bool PASS>
-bool launch_scan_rows(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
+bool launch_scan_rows(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaStream_t stream, bool pdl) {
+  const dim3 block(kScanThreads);
   if (esize == 1 && lpr == 8)
-    decode_scan_rows_kernel<1, 8, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_maybe_programmatic(decode_scan_rows_kernel<1, 8, PAGED, NQ, PASS>, grid, block, 0, stream, pdl, sp);
   else if (esize == 1 && lpr == 4)
-    decode_scan_rows_kernel<1, 4, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_maybe_programmatic(decode_scan_rows_kernel<1, 4, PAGED, NQ, PASS>, grid, block, 0, stream, pdl, sp);
   else if (esize == 1 && lpr == 16)
-    decode_scan_rows_kernel<1, 16, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_maybe_programmatic(decode_scan_rows_kernel<1, 16, PAGED, NQ, PASS>, grid, block, 0, stream, pdl, sp);
   else if (esize == 2 && lpr == 8)
-    decode_scan_rows_kernel<2, 8, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_maybe_programmatic(decode_scan_rows_kernel<2, 8, PAGED, NQ, PASS>, grid, block, 0, stream, pdl, sp);
   else if (esize == 2 && lpr == 16)
-    decode_scan_rows_kernel<2, 16, PAGED, NQ, PASS><<<grid, kScanThreads, 0, stream>>>(sp);
+    launch_maybe_programmatic(decode_scan_rows_kernel<2, 16, PAGED, NQ, PASS>, grid, block, 0, stream, pdl, sp);
   else
     return false;
   return true;
@@ -693,19 +699,19 @@ bool launch_scan_rows(const ScanParams& sp, dim3 grid, int esize, int lpr, cudaS
 template <bool PAGED>
 bool launch_scan(ScanParams sp, dim3 grid, int esize, int lpr, cudaStream_t stream) {
   sp.q_first = 0;
-  if (sp.nq == 2) return launch_scan_rows<PAGED, 2, false>(sp, grid, esize, lpr, stream);
+  if (sp.nq == 2) return launch_scan_rows<PAGED, 2, false>(sp, grid, esize, lpr, stream, true);
   if (sp.nq == 1) {
-    if (launch_scan_rows<PAGED, 1, false>(sp, grid, esize, lpr, stream)) return true;
+    if (launch_scan_rows<PAGED, 1, false>(sp, grid, esize, lpr, stream, true)) return true;
     if (esize == 1)
-      decode_scan_kernel<1, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+      launch_maybe_programmatic(decode_scan_kernel<1, PAGED>, grid, dim3(kScanThreads), 0, stream, true, sp);
     else
-      decode_scan_kernel<2, PAGED><<<grid, kScanThreads, 0, stream>>>(sp);
+      launch_maybe_programmatic(decode_scan_kernel<2, PAGED>, grid, dim3(kScanThreads), 0, stream, true, sp);
     return true;
   }
   for (int q = 0; q < sp.nq; q += 2) {
     sp.q_first = q;
-    const bool ok = q + 1 < sp.nq ? launch_scan_rows<PAGED, 2, true>(sp, grid, esize, lpr, stream)
-                                  : launch_scan_rows<PAGED, 1, true>(sp, grid, esize, lpr, stream);
+    const bool ok = q + 1 < sp.nq ? launch_scan_rows<PAGED, 2, true>(sp, grid, esize, lpr, stream, q == 0)
+                                  : launch_scan_rows<PAGED, 1, true>(sp, grid, esize, lpr, stream, q == 0);
     if (!ok) return false;
   }
   return true;
