@@ -642,6 +642,43 @@ def run_decode_paged(dsa, xp, top_k, max_len=None):
     return idx, O
 
 
+def test_decode_with_stage_timing_matches_plain_calls(dsa):
+    """The decode kernels follow one another by programmatic launches; stage
+    timing records CUDA events between them.  Results with and without the
+    events must be identical (contiguous, paged and two-token steps), and the
+    decode stages must be timed."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([2, 100, 2049, 9000, 70000], dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    xp = synth.paged_decode_inputs(w, lens, 64)
+    mq = synth.multi_queries(w, len(lens), 2)
+    t = {k: to_dev(xd[k]) for k in ("k_idx", "K", "V", "seq_start")}
+    tm = {k: to_dev(mq[k]) for k in ("q_idx", "Q")}
+
+    def calls():
+        a = run_decode(dsa, xd, w.top_k)
+        idx, O = run_decode_paged(dsa, xp, w.top_k)
+        b = (idx.cpu().numpy(), O.view(torch.int16).cpu().numpy())
+        O2, idx2 = dsa.dsa_decode_multi(t["k_idx"], t["K"].view(torch.bfloat16), t["V"].view(torch.bfloat16),
+                                        t["seq_start"], tm["q_idx"], tm["Q"].view(torch.bfloat16), w.top_k,
+                                        int(lens.max()))
+        assert dsa.dsa_sync_status() == 0
+        return a + b + (idx2.cpu().numpy(), O2.view(torch.int16).cpu().numpy())
+
+    plain = calls()
+    dsa.dsa_stage_times()   # reset
+    dsa.dsa_stage_timing(True)
+    try:
+        timed = calls()
+        times = dsa.dsa_stage_times()
+    finally:
+        dsa.dsa_stage_timing(False)
+    for x, y in zip(plain, timed):
+        assert np.array_equal(x, y)
+    assert times["decode_scan_select"][1] > 0 and times["decode_scan_select"][0] > 0
+    assert times["decode_attention"][1] > 0 and times["decode_attention"][0] > 0
+
+
 @pytest.mark.parametrize("block_size,idx_dtype,d,D,top_k", [
     (1, "fp8", 128, 128, 256),       # one row per block
     (16, "fp8", 128, 128, 2048),
