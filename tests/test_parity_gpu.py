@@ -642,6 +642,57 @@ def run_decode_paged(dsa, xp, top_k, max_len=None):
     return idx, O
 
 
+def test_decode_step_replays_from_a_cuda_graph(dsa):
+    """A decode step (memsets and programmatically launched kernels) captured in
+    a CUDA graph replays to the results of an ordinary call, contiguous and
+    paged cache."""
+    w = synth.WORKLOADS["decode_64x128k"]
+    lens = np.array([2, 100, 2049, 9000, 70000], dtype=np.int64)
+    xd = synth.decode_inputs(w, lengths=lens)
+    xp = synth.paged_decode_inputs(w, lens, 64)
+    t = {k: to_dev(xd[k]) for k in ("k_idx", "K", "V", "q_idx", "Q", "seq_start")}
+    tp = {k: to_dev(xp[k]) for k in ("k_idx_blocks", "K_blocks", "V_blocks", "block_table", "seq_lens",
+                                     "q_idx", "Q")}
+    B, mx = len(lens), int(lens.max())
+    O = torch.empty((B, w.H, w.D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.empty((B, w.top_k), dtype=torch.int32, device="cuda")
+    Op, idxp = torch.empty_like(O), torch.empty_like(idx)
+    ws = torch.empty(dsa.dsa_decode_workspace_size(B, int(lens.sum()), w.d_idx, 0, w.H, w.D, w.top_k),
+                     dtype=torch.uint8, device="cuda")
+    wsp = torch.empty(dsa.dsa_decode_paged_workspace_size(B, mx, w.d_idx, 0, w.H, w.D, w.top_k),
+                      dtype=torch.uint8, device="cuda")
+
+    def step():
+        dsa.dsa_decode(t["k_idx"], t["K"].view(torch.bfloat16), t["V"].view(torch.bfloat16), t["seq_start"],
+                       t["q_idx"], t["Q"].view(torch.bfloat16), w.top_k, mx, O=O, indices=idx, workspace=ws)
+        dsa.dsa_decode_paged(tp["k_idx_blocks"], tp["K_blocks"].view(torch.bfloat16),
+                             tp["V_blocks"].view(torch.bfloat16), tp["block_table"], tp["seq_lens"],
+                             tp["q_idx"], tp["Q"].view(torch.bfloat16), w.top_k, mx, O=Op, indices=idxp,
+                             workspace=wsp)
+
+    step()
+    torch.cuda.synchronize()
+    assert dsa.dsa_sync_status() == 0
+    ref = [x.clone() for x in (idx, O, idxp, Op)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for x in (idx, O, idxp, Op):
+        x.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert dsa.dsa_sync_status() == 0
+    for x, y in zip((idx, O, idxp, Op), ref):
+        assert torch.equal(x.view(torch.int16) if x.dtype == torch.bfloat16 else x,
+                           y.view(torch.int16) if y.dtype == torch.bfloat16 else y)
+    del g
+
+
 def test_decode_with_stage_timing_matches_plain_calls(dsa):
     """The decode kernels follow one another by programmatic launches; stage
     timing records CUDA events between them.  Results with and without the
