@@ -642,6 +642,48 @@ def run_decode_paged(dsa, xp, top_k, max_len=None):
     return idx, O
 
 
+@pytest.mark.parametrize("idx_dtype,d,H,D,top_k", [("bf16", 160, 16, 128, 2048), ("fp8", 128, 4, 64, 256)])
+def test_prefill_step_replays_from_a_cuda_graph(dsa, idx_dtype, d, H, D, top_k):
+    """A prefill step (threshold sample, filter, select with its queued large-row
+    and fallback passes, attention) captured in a CUDA graph replays to the
+    results of an ordinary call: every decision between the kernels is taken on
+    the device."""
+    L = 5000
+    x = small_inputs(L, d, H, D, idx_dtype)
+    q, k = to_dev(x["q_idx"]), to_dev(x["k_idx"])
+    if q.dtype == torch.uint16:
+        q, k = q.view(torch.bfloat16), k.view(torch.bfloat16)
+    Q, K, V = bf16(x["Q"]), bf16(x["K"]), bf16(x["V"])
+    ws = torch.empty(dsa.dsa_prefill_workspace_size(L, d, 0 if idx_dtype == "fp8" else 1, H, D, top_k),
+                     dtype=torch.uint8, device="cuda")
+    idx = torch.empty((L, top_k), dtype=torch.int32, device="cuda")
+    O = torch.empty((L, H, D), dtype=torch.bfloat16, device="cuda")
+
+    def step():
+        dsa.dsa_prefill(q, k, Q, K, V, top_k, indices=idx, O=O, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    assert dsa.dsa_sync_status() == 0
+    ref_idx, ref_o = idx.clone(), O.clone()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    idx.zero_()
+    O.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert dsa.dsa_sync_status() == 0
+    assert torch.equal(idx, ref_idx)
+    assert torch.equal(O.view(torch.int16), ref_o.view(torch.int16))
+    del g
+
+
 def test_decode_step_replays_from_a_cuda_graph(dsa):
     """A decode step (memsets and programmatically launched kernels) captured in
     a CUDA graph replays to the results of an ordinary call, contiguous and
