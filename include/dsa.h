@@ -30,7 +30,12 @@
  *     128-byte alignment is recommended (row starts then fall on 128 B).
  *   - `stream` is a cudaStream_t passed as void*.  Calls only enqueue work;
  *     they are asynchronous and keep no state between calls, so calls on
- *     distinct workspaces may run concurrently.
+ *     distinct workspaces may run concurrently.  No compute call synchronises
+ *     with the host (only dsa_sync_status, dsa_last_stats and
+ *     dsa_stage_times do), so after one ordinary call with the same shapes
+ *     (which loads the kernels) a dsa_prefill* or dsa_decode* call with a
+ *     caller's workspace may be captured into a CUDA graph and replayed with
+ *     the same pointers and sizes.
  *   - Argument errors are reported synchronously by the return value and
  *     nothing is enqueued.  Errors found on the device (a bounded wait that
  *     ran out; decode lengths or block ids that fail the device-side checks)
